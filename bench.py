@@ -1,0 +1,371 @@
+"""Benchmark of the verified sparse decode step (vattn_decode) on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload gqa_32k] [--eps E]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+One step = one vattn_decode call over the whole batch of the workload (every
+row of the hot path: query prep, ranking-score pass, top-k select, pilot,
+budget, gather, combine). Inputs are resident in HBM before the timed region
+and larger than L2 (so no flush is needed). Prints one JSON line (rank 0).
+Under torchrun each rank runs its own batch on its own GPU (weak scaling; no
+collective on the data path, one max-reduction of the elapsed time).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from verified_sparse_attention_b200 import _abi, synth  # noqa: E402
+from verified_sparse_attention_b200.decoder import decoder_for, params_for  # noqa: E402
+
+METRIC = "sparse decode-attn calls/s & achieved HBM GB/s (% of ~8 TB/s) at 32k–128k ctx"
+KERNEL_SOURCES = ["verified_sparse_attention_b200/csrc/vattn_kernels.cuh",
+                  "verified_sparse_attention_b200/csrc/vattn_device.cuh"]
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per score-pass launch from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", f"score_pass_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_hash") != kernel_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """SM clock and throttle reasons sampled through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.ok = period, False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            get = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            r = get(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ byte accounting
+def algorithmic_bytes(w, x, res):
+    """(score-pass bytes per launch, whole-call KV bytes) from the call's own outputs."""
+    e = synth.bytes_per_elem(w)
+    d = w.head_dim
+    n = x["seq_lens"].to(torch.int64).cpu()
+    s1 = torch.clamp(n, max=w.sinks)
+    wst = torch.maximum(n - w.window, s1)
+    mid = (wst - s1).clamp(min=0)                          # middle rows per sequence
+    per_row = {"exact": d * e, "sparq": w.proxy_rank * e, "loki": w.proxy_rank * e}[w.proxy]
+    score = int(mid.sum()) * w.num_kv_heads * (per_row + 4)     # K (or proxy) read + key write
+    cnt = res["sel_count"].to(torch.int64).cpu()            # [B, Hkv] rows gathered (K and V)
+    gather = int(cnt.sum()) * 2 * d * e
+    return score, score + gather
+
+
+# ------------------------------------------------------------------ arms
+def run_gpu_arm(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    if rank:
+        w = w.replace(data_seed=w.data_seed + 1000 * rank)
+    x = synth.make_inputs(w, device=dev)
+    dec = decoder_for(w, device=dev)
+    prm = params_for(w, x, eps=args.eps)
+    outs = dec.alloc_outputs(w.batch)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dec.decode(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"], prm,
+                   outputs=outs, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dec.last_error():
+        raise RuntimeError("device error word set during warm-up")
+    launches_per_call = _abi.vattn_last_launch_count(dec.ctx)
+    _abi.vattn_score_pass_ms(dec.ctx, reset=True)
+    _abi.vattn_set_timing(dec.ctx, True)
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    _abi.vattn_set_timing(dec.ctx, False)
+    ms = t0.elapsed_time(t1)
+    score_ms, score_n = _abi.vattn_score_pass_ms(dec.ctx, reset=True)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    score_bytes, call_bytes = algorithmic_bytes(w, x, outs)
+    budgets = outs["budgets"].cpu()
+
+    # dense decode attention on the same inputs (comparison baseline)
+    for _ in range(args.warmup):
+        dec.dense(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"],
+                  x["num_pages"], stream=stream)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(args.steps):
+        dec.dense(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"],
+                  x["num_pages"], stream=stream)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / args.steps
+
+    e2e = run_e2e(args, w, x, dec, prm, stream, dev, world)
+
+    result = dict(w=w, x=x, ms=ms_max, score_ms=score_ms, score_n=score_n,
+                  score_bytes=score_bytes, call_bytes=call_bytes, budgets=budgets,
+                  launches=launches_per_call * args.steps, clocks=clk.summary(),
+                  dense_ms=dense_ms, e2e=e2e)
+    return dec, result
+
+
+def run_e2e(args, w, x, dec, prm, stream, dev, world):
+    """Same metric through the C ABI with host buffers: pinned host -> device copies of
+    every input and a device -> host read of the result inside the timed region."""
+    keys = ["q", "k_cache", "v_cache", "page_table", "seq_lens"]
+    extra = [k for k in ("k_t_cache", "k_proj_cache", "proj_basis") if k in x]
+    host = {k: x[k].cpu().pin_memory() for k in keys + extra}
+    devb = {k: torch.empty_like(x[k]) for k in keys + extra}
+    outs = dec.alloc_outputs(w.batch)
+    out_h = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+             for k, v in outs.items() if k != "sel_idx"}
+    p = params_for(w, {**devb, "num_pages": x["num_pages"]}, eps=args.eps)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_h.values())
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        for k in host:
+            devb[k].copy_(host[k], non_blocking=True)
+        dec.decode(devb["q"], devb["k_cache"], devb["v_cache"], devb["page_table"],
+                   devb["seq_lens"], p, outputs=outs, stream=stream)
+        for k in out_h:
+            out_h[k].copy_(outs[k], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    del devb, host
+    return {"value": world * steps / (ms / 1e3), "unit": "calls/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def time_oracle(w, cpu_inputs, budget_s, units_per_step=None):
+    """Run the oracle unit by unit on the host until budget_s elapses (or all units).
+    Returns (calls/s equivalent, units done, seconds)."""
+    import oracle
+    pr = oracle.make_problem(w)
+    U = w.units
+    done, t0 = 0, time.perf_counter()
+    u = 0
+    while True:
+        oracle.decode(pr, cpu_inputs, units=[u % U])
+        done += 1
+        u += 1
+        el = time.perf_counter() - t0
+        if units_per_step is not None and done >= units_per_step:
+            break
+        if units_per_step is None and (el >= budget_s or done >= 5 * U):
+            break
+    el = time.perf_counter() - t0
+    return (done / U) / el, done, el
+
+
+def emit(line):
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gqa_32k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--eps", type=float, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    if args.eps is not None:
+        w = w.replace(eps=args.eps)
+    cfg = {"workload": synth.describe(w), "name": w.name, "batch": w.batch,
+           "ctx": w.max_ctx if w.min_ctx == w.max_ctx else [w.min_ctx, w.max_ctx],
+           "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        t_gen = time.perf_counter()
+        cpu = synth.make_inputs(w)
+        gen_s = time.perf_counter() - t_gen
+        ups = max(1, w.units // 16)
+        for _ in range(args.warmup):
+            time_oracle(w, cpu, 0, units_per_step=1)
+        t0 = time.perf_counter()
+        done = 0
+        for _ in range(args.steps):
+            _, d, _ = time_oracle(w, cpu, 0, units_per_step=ups)
+            done += d
+        el = time.perf_counter() - t0
+        val = (done / w.units) / el
+        emit({"impl": "reference", "metric": METRIC, "value": val, "unit": "calls/s",
+              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+              "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+              "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
+              "cpu_baseline": {"value": val, "unit": "calls/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{ups} of {w.units} (sequence, KV head) units per step, "
+                                         f"single-threaded C oracle; input generation {gen_s:.1f}s untimed"},
+              "e2e": {"value": val, "unit": "calls/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dec, r = run_gpu_arm(args, rank, world, local_rank)
+    peak, peak_kind = load_peaks()
+    w = r["w"]
+    calls_s = world * args.steps / (r["ms"] / 1e3)
+    avg_score_s = (r["score_ms"] / max(1, r["score_n"])) / 1e3
+    achieved = r["score_bytes"] / avg_score_s / 1e9
+    call_s = r["ms"] / 1e3 / args.steps
+    line = {"metric": METRIC, "value": calls_s, "unit": "calls/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic", "config": cfg,
+            "roofline": {"bound": "hbm", "kernel": "score pass (k_score_rows / k_score_sparq)",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": profiled_traffic(w.name),
+                         "algorithmic_bytes_per_launch": r["score_bytes"],
+                         "avg_launch_us": avg_score_s * 1e6},
+            "call_kv_bytes": r["call_bytes"],
+            "call_achieved_gbs": r["call_bytes"] / call_s / 1e9,
+            "call_frac_of_peak": r["call_bytes"] / call_s / 1e9 / peak,
+            "dense_calls_per_s": world / (r["dense_ms"] / 1e3),
+            "budget_mean": float(r["budgets"].float().mean()),
+            "gpu_launches": r["launches"], "clocks": r["clocks"], "e2e": r["e2e"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in r["x"].items()}
+        val, done, el = time_oracle(w, cpu, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": val, "unit": "calls/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{done} (sequence, KV head) units of a {w.units}-unit call "
+                                          f"in {el:.1f}s, single-threaded C oracle"}
+    dec.close()
+    if rank == 0:
+        emit(line)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

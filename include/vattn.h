@@ -1,0 +1,159 @@
+/*
+ * vattn — verified sparse attention (vAttention) for one decode step, on
+ * B200 (sm_100a).
+ *
+ * The operation (from "vAttention: A New Approach to Sparse Attention with
+ * Guaranteed Accuracy", section "How vAttention Works", and the paragraph
+ * after it on the denominator): for every sequence b and KV head h of a
+ * decode step, attention over the cached keys is approximated by
+ *   - a deterministic index set I_f: the first `sinks` positions (attention
+ *     sinks), the last `window` positions (sliding window) and the top-k of
+ *     the remaining middle positions under a ranking score (predicted top-k);
+ *   - a uniform random sample, with replacement, of the remaining tail T,
+ *     |T| = N_tail, whose size b is set from a pilot sample by the Central
+ *     Limit Theorem: n >= (z_{1-delta/2} * N_tail * sigma / (eps * D))^2, so
+ *     that the softmax denominator D has relative error <= eps with
+ *     probability about 1 - delta;
+ *   - output o = (A_f + (N_tail/b) A_s) / (L_f + (N_tail/b) L_s), where A and
+ *     L are the exp-weighted value sums and exp sums over I_f and the sample.
+ * The ranking score is exact (q . k), a SparQ-style proxy over the r largest
+ * query components ("SparQ Attention: Bandwidth-Efficient LLM Inference",
+ * abstract), or a Loki-style score in a stored low-rank key space ("Loki:
+ * Low-rank Keys for Efficient Sparse Attention", abstract).
+ *
+ * Memory: every array argument is caller-owned DEVICE memory unless stated;
+ * the context owns only its workspace, allocated once in vattn_create.
+ * vattn_decode allocates nothing, never synchronises the host, and enqueues
+ * all its work on `stream`, so it may be captured in a CUDA graph.
+ *
+ * Layouts (row-major, innermost last; Hq query heads, Hkv KV heads, d head
+ * dim, G = Hq/Hkv, query head hq belongs to KV head hq / G):
+ *   q          [batch][Hq][d]                       dtype
+ *   k_cache    [num_pages][Hkv][page_size][d]       dtype
+ *   v_cache    [num_pages][Hkv][page_size][d]       dtype
+ *   page_table [batch][pages_per_seq] int32, pages_per_seq = ceil(max_ctx/page_size);
+ *              entries for positions < seq_lens[b] must lie in [0, num_pages)
+ *   seq_lens   [batch] int32, 0 <= seq_lens[b] <= max_ctx
+ *   out        [batch][Hq][d] float32
+ *   sel_idx    [batch][Hkv][max_ctx] int32: I_f ascending, then the b sample
+ *              positions in draw order (repeats kept), or, when the sample
+ *              would cover the tail (b >= N_tail), the whole tail ascending
+ *   sel_count  [batch][Hkv] int32: |I_f| + b (or + N_tail)
+ *   budgets    [batch][Hkv] int32: b (N_tail when the tail was taken whole,
+ *              0 when there is no tail)
+ *   head_need  [batch][Hq] int32: n_h, the CLT size required by query head
+ *              hq (N_tail when the tail was taken whole before any pilot)
+ * A contiguous cache is one page per sequence: page_size = max_ctx (a power
+ * of two) and page_table[b][0] = b.
+ *
+ * Return codes: VATTN_OK, or a negative VATTN_E* code for bad host arguments
+ * (nothing is launched) or a CUDA launch failure. Device-side violations (a
+ * page id out of range, a sequence length outside [0, max_ctx]) never trap:
+ * the kernel treats that sequence as empty (zero output, empty selection)
+ * and sets a bit in the context's device error word, read by
+ * vattn_last_error.
+ */
+#ifndef VATTN_H
+#define VATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { VATTN_FP32 = 0, VATTN_BF16 = 1 };
+enum { VATTN_EXACT = 0, VATTN_SPARQ = 1, VATTN_LOKI = 2 };
+
+enum {
+  VATTN_OK = 0,
+  VATTN_EINVAL = -1, /* a host argument is out of range or a required pointer is NULL */
+  VATTN_ENOMEM = -2, /* workspace allocation failed in vattn_create                 */
+  VATTN_ECUDA = -3   /* a CUDA call or kernel launch failed                          */
+};
+
+/* bits of the device error word */
+enum { VATTN_DEV_BAD_SEQLEN = 1, VATTN_DEV_BAD_PAGE = 2 };
+
+typedef struct vattn_ctx vattn_ctx;
+
+/* Fixed for the life of a context. */
+typedef struct {
+  int num_q_heads;  /* Hq, a multiple of num_kv_heads with Hq/Hkv in {1,2,4,8} */
+  int num_kv_heads; /* Hkv >= 1                                                  */
+  int head_dim;     /* d in {64, 128}                                            */
+  int dtype;        /* VATTN_FP32 or VATTN_BF16, for q and every cache          */
+  int page_size;    /* power of two >= 16 (contiguous cache: = max_ctx)          */
+  int max_batch;    /* upper bound on `batch` in every call                      */
+  int max_ctx;      /* upper bound on seq_lens[b]; 1 <= max_ctx <= 2^24          */
+  int proxy;        /* VATTN_EXACT, VATTN_SPARQ or VATTN_LOKI                    */
+  int proxy_rank;   /* SparQ: r in [1, d]; Loki: the stored rank, 32             */
+} vattn_config;
+
+/* Per call. */
+typedef struct {
+  int sinks, window; /* >= 0                                                      */
+  /* top-k size for a sequence of length N: topk_abs if topk_den == 0, else
+     floor(N * topk_num / topk_den); then capped by the middle's length        */
+  int topk_abs, topk_num, topk_den;
+  /* pilot size: pilot_min if pilot_den == 0, else
+     max(pilot_min, ceil(N * pilot_num / pilot_den)); pilot_min >= 2           */
+  int pilot_min, pilot_num, pilot_den;
+  float eps;         /* > 0: relative error target on the softmax denominator   */
+  float delta;       /* in (0, 1): allowed failure probability                  */
+  uint64_t seed;     /* Philox4x32-10 key of the tail sampler                   */
+  int num_pages;     /* pages in the caches (bound for page_table entries)      */
+  const void* k_t_cache;    /* SparQ: dim-major K [num_pages][Hkv][d][page_size], else NULL  */
+  const void* k_proj_cache; /* Loki: projected K [num_pages][Hkv][page_size][rank], else NULL */
+  const float* proj_basis;  /* Loki: basis fp32 [Hkv][d][rank], else NULL                     */
+} vattn_params;
+
+/* Create a context on the current CUDA device and allocate its workspace.
+   Returns VATTN_OK and sets *out, or VATTN_EINVAL / VATTN_ENOMEM. */
+int vattn_create(vattn_ctx** out, const vattn_config* cfg);
+
+/* One sparse decode step (the operation described above) for `batch`
+   sequences, enqueued on `stream` (a cudaStream_t; NULL = legacy default). */
+int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* page_table, const int32_t* seq_lens, int batch,
+                 const vattn_params* params, float* out, int32_t* sel_idx, int32_t* sel_count,
+                 int32_t* budgets, int32_t* head_need, void* stream);
+
+/* Dense decode attention over all seq_lens[b] positions, same layouts: the
+   comparison baseline for vattn_decode (softmax(q K^T / sqrt(d)) V). */
+int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* seq_lens, int batch,
+                       int num_pages, float* out, void* stream);
+
+/* sync != 0: wait for the device, then return and clear the device error
+   word (VATTN_DEV_* bits). sync == 0: return the host status of the last
+   call on this context, without touching the device. */
+int vattn_last_error(vattn_ctx* ctx, int sync);
+
+/* Bytes of device workspace the context holds. */
+size_t vattn_workspace_bytes(const vattn_ctx* ctx);
+
+/* Per-call kernel timing: when enabled, vattn_decode records a CUDA event
+   pair around its dominant kernel (the ranking-score pass) on `stream`;
+   vattn_score_pass_ms returns the summed elapsed time in milliseconds since
+   the last reset and how many passes it covers. Calls synchronise on the
+   recorded events (host wait). */
+int vattn_set_timing(vattn_ctx* ctx, int enable);
+int vattn_score_pass_ms(vattn_ctx* ctx, double* total_ms, int* count, int reset);
+
+/* Number of kernel launches the last vattn_decode / vattn_dense_decode call
+   enqueued. */
+int vattn_last_launch_count(const vattn_ctx* ctx);
+
+/* Text for a return code. */
+const char* vattn_strerror(int code);
+
+/* Release the workspace and the context. NULL is allowed. */
+void vattn_destroy(vattn_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VATTN_H */

@@ -1,0 +1,460 @@
+// Host side of the C ABI declared in include/vattn.h: argument checks,
+// workspace, template dispatch and the launch sequence of one decode step.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "vattn.h"
+#include "vattn_kernels.cuh"
+
+using vattn::DevParams;
+using vattn::UnitInfo;
+
+struct vattn_ctx {
+  vattn_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  int G = 1;
+  int units_max = 0;
+  int nseg = 0;
+  int score_grid = 0;
+  int gather_occ = 1;
+  size_t ws_bytes = 0;
+  void* ws = nullptr;
+  // carved workspace
+  UnitInfo* info = nullptr;
+  float* qbar = nullptr;
+  float* qsel = nullptr;
+  int* dims = nullptr;
+  unsigned* ordk = nullptr;
+  unsigned* hist = nullptr;
+  unsigned* segcnt = nullptr;
+  float* pscore = nullptr;
+  float* partial = nullptr;
+  long long* prefix = nullptr;
+  unsigned* err = nullptr;
+  // state
+  int last_status = VATTN_OK;
+  int last_launches = 0;
+  double cached_delta = -1.0;
+  double cached_z = 0.0;
+  // timing of the score pass
+  int timing = 0;
+  std::vector<cudaEvent_t> ev_start, ev_stop;
+  size_t ev_used = 0;
+};
+
+namespace {
+
+// z_{1-delta/2}: 200 bisection steps on [0, 40] of the upper normal tail
+// 0.5 * erfc(z / sqrt 2) against delta / 2.
+double normal_upper_quantile(double delta) {
+  double lo = 0.0, hi = 40.0;
+  const double target = 0.5 * delta;
+  for (int it = 0; it < 200; it++) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * erfc(mid * 0.70710678118654752440) > target)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int log2i(int x) {
+  int r = 0;
+  while ((1 << r) < x) r++;
+  return r;
+}
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- dispatch
+struct Kernels {
+  void (*prep)(DevParams);
+  void (*score_exact)(DevParams);
+  void (*score_loki)(DevParams);
+  void (*score_sparq)(DevParams);
+  void (*pilot)(DevParams);
+  void (*budget)(DevParams);
+  void (*gather)(DevParams);
+  void (*combine)(DevParams);
+};
+
+template <typename T, int D, int G>
+Kernels kernels_for() {
+  Kernels k;
+  k.prep = vattn::k_prep<T, D, G>;
+  k.score_exact = vattn::k_score_rows<T, D>;
+  k.score_loki = vattn::k_score_rows<T, 32>;
+  k.score_sparq = vattn::k_score_sparq<T, D>;
+  k.pilot = vattn::k_pilot<T, D, G>;
+  k.budget = vattn::k_budget<G>;
+  k.gather = vattn::k_gather<T, D, G>;
+  k.combine = vattn::k_combine<D, G>;
+  return k;
+}
+
+template <typename T, int D>
+bool pick_g(int G, Kernels* k) {
+  switch (G) {
+    case 1: *k = kernels_for<T, D, 1>(); return true;
+    case 2: *k = kernels_for<T, D, 2>(); return true;
+    case 4: *k = kernels_for<T, D, 4>(); return true;
+    case 8: *k = kernels_for<T, D, 8>(); return true;
+    default: return false;
+  }
+}
+
+bool pick(const vattn_config& c, int G, Kernels* k) {
+  if (c.dtype == VATTN_BF16) {
+    if (c.head_dim == 128) return pick_g<__nv_bfloat16, 128>(G, k);
+    if (c.head_dim == 64) return pick_g<__nv_bfloat16, 64>(G, k);
+  } else if (c.dtype == VATTN_FP32) {
+    if (c.head_dim == 128) return pick_g<float, 128>(G, k);
+    if (c.head_dim == 64) return pick_g<float, 64>(G, k);
+  }
+  return false;
+}
+
+int check_config(const vattn_config* c) {
+  if (!c) return VATTN_EINVAL;
+  if (c->num_kv_heads < 1 || c->num_q_heads < 1 || c->num_q_heads % c->num_kv_heads) return VATTN_EINVAL;
+  const int G = c->num_q_heads / c->num_kv_heads;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8)) return VATTN_EINVAL;
+  if (!(c->head_dim == 64 || c->head_dim == 128)) return VATTN_EINVAL;
+  if (!(c->dtype == VATTN_FP32 || c->dtype == VATTN_BF16)) return VATTN_EINVAL;
+  if (!is_pow2(c->page_size) || c->page_size < 16) return VATTN_EINVAL;
+  if (c->max_batch < 1 || c->max_ctx < 1 || c->max_ctx > (1 << 24)) return VATTN_EINVAL;
+  if (c->proxy == VATTN_SPARQ) {
+    if (c->proxy_rank < 1 || c->proxy_rank > c->head_dim) return VATTN_EINVAL;
+  } else if (c->proxy == VATTN_LOKI) {
+    if (c->proxy_rank != 32) return VATTN_EINVAL;
+  } else if (c->proxy != VATTN_EXACT) {
+    return VATTN_EINVAL;
+  }
+  return VATTN_OK;
+}
+
+void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
+  memset(P, 0, sizeof(*P));
+  const vattn_config& c = ctx->cfg;
+  P->Hq = c.num_q_heads;
+  P->Hkv = c.num_kv_heads;
+  P->G = ctx->G;
+  P->D = c.head_dim;
+  P->pps = (c.max_ctx + c.page_size - 1) / c.page_size;
+  P->ps_log2 = log2i(c.page_size);
+  P->max_ctx = c.max_ctx;
+  P->batch = batch;
+  P->units = batch * c.num_kv_heads;
+  P->proxy = c.proxy;
+  P->rank = c.proxy_rank;
+  P->scale = static_cast<float>(1.0 / sqrt(static_cast<double>(c.head_dim)));
+  P->nseg = ctx->nseg;
+  P->info = ctx->info;
+  P->qbar = ctx->qbar;
+  P->qsel = ctx->qsel;
+  P->dims = ctx->dims;
+  P->ordk = ctx->ordk;
+  P->hist = ctx->hist;
+  P->segcnt = ctx->segcnt;
+  P->pscore = ctx->pscore;
+  P->partial = ctx->partial;
+  P->prefix = ctx->prefix;
+  P->err = ctx->err;
+}
+
+int splits_for(int want, int units) {
+  int s = (want + units - 1) / units;
+  if (s < 1) s = 1;
+  if (s > vattn::kSbMax) s = vattn::kSbMax;
+  return s;
+}
+
+int finish(vattn_ctx* ctx, int launches) {
+  ctx->last_launches = launches;
+  const cudaError_t e = cudaGetLastError();
+  ctx->last_status = e == cudaSuccess ? VATTN_OK : VATTN_ECUDA;
+  return ctx->last_status;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vattn_strerror(int code) {
+  switch (code) {
+    case VATTN_OK: return "ok";
+    case VATTN_EINVAL: return "invalid argument";
+    case VATTN_ENOMEM: return "device workspace allocation failed";
+    case VATTN_ECUDA: return "CUDA call or kernel launch failed";
+    default: return "unknown code";
+  }
+}
+
+int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
+  if (!out) return VATTN_EINVAL;
+  *out = nullptr;
+  if (check_config(cfg) != VATTN_OK) return VATTN_EINVAL;
+  vattn_ctx* ctx = new vattn_ctx();
+  ctx->cfg = *cfg;
+  ctx->G = cfg->num_q_heads / cfg->num_kv_heads;
+  Kernels K;
+  if (!pick(ctx->cfg, ctx->G, &K)) {
+    delete ctx;
+    return VATTN_EINVAL;
+  }
+  if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
+    delete ctx;
+    return VATTN_ECUDA;
+  }
+  const int D = cfg->head_dim, G = ctx->G;
+  const size_t U = static_cast<size_t>(cfg->max_batch) * cfg->num_kv_heads;
+  ctx->units_max = static_cast<int>(U);
+  ctx->nseg = (cfg->max_ctx + vattn::kSeg - 1) / vattn::kSeg;
+  const size_t sz_info = align256(U * sizeof(UnitInfo));
+  const size_t sz_vec = align256(U * D * sizeof(float));
+  const size_t sz_ordk = align256(U * cfg->max_ctx * sizeof(unsigned));
+  const size_t sz_hist = align256(U * vattn::kHistAll * sizeof(unsigned));
+  const size_t sz_seg = align256(U * ctx->nseg * 2 * sizeof(unsigned));
+  const size_t sz_ps = align256(U * cfg->max_ctx * G * sizeof(float));
+  const size_t sz_part = align256(U * vattn::kSbMax * G * (4 + 2 * D) * sizeof(float));
+  const size_t sz_pre = align256((U + 1) * sizeof(long long));
+  const size_t sz_err = 256;
+  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_part + sz_pre + sz_err;
+  if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete ctx;
+    return VATTN_ENOMEM;
+  }
+  char* p = static_cast<char*>(ctx->ws);
+  ctx->info = reinterpret_cast<UnitInfo*>(p); p += sz_info;
+  ctx->qbar = reinterpret_cast<float*>(p); p += sz_vec;
+  ctx->qsel = reinterpret_cast<float*>(p); p += sz_vec;
+  ctx->dims = reinterpret_cast<int*>(p); p += sz_vec;
+  ctx->ordk = reinterpret_cast<unsigned*>(p); p += sz_ordk;
+  ctx->hist = reinterpret_cast<unsigned*>(p); p += sz_hist;
+  ctx->segcnt = reinterpret_cast<unsigned*>(p); p += sz_seg;
+  ctx->pscore = reinterpret_cast<float*>(p); p += sz_ps;
+  ctx->partial = reinterpret_cast<float*>(p); p += sz_part;
+  ctx->prefix = reinterpret_cast<long long*>(p); p += sz_pre;
+  ctx->err = reinterpret_cast<unsigned*>(p);
+  if (cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess) {
+    cudaFree(ctx->ws);
+    delete ctx;
+    return VATTN_ECUDA;
+  }
+  void (*score)(DevParams) = cfg->proxy == VATTN_SPARQ ? K.score_sparq
+                             : cfg->proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
+  if (occ < 1) occ = 1;
+  ctx->score_grid = occ * ctx->num_sms;
+  int gocc = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.gather, 256, 0);
+  ctx->gather_occ = gocc < 1 ? 1 : gocc;
+  if (cudaGetLastError() != cudaSuccess) {
+    cudaFree(ctx->ws);
+    delete ctx;
+    return VATTN_ECUDA;
+  }
+  *out = ctx;
+  return VATTN_OK;
+}
+
+void vattn_destroy(vattn_ctx* ctx) {
+  if (!ctx) return;
+  for (auto e : ctx->ev_start) cudaEventDestroy(e);
+  for (auto e : ctx->ev_stop) cudaEventDestroy(e);
+  if (ctx->ws) cudaFree(ctx->ws);
+  delete ctx;
+}
+
+size_t vattn_workspace_bytes(const vattn_ctx* ctx) { return ctx ? ctx->ws_bytes : 0; }
+
+int vattn_last_launch_count(const vattn_ctx* ctx) { return ctx ? ctx->last_launches : 0; }
+
+int vattn_set_timing(vattn_ctx* ctx, int enable) {
+  if (!ctx) return VATTN_EINVAL;
+  ctx->timing = enable ? 1 : 0;
+  return VATTN_OK;
+}
+
+int vattn_score_pass_ms(vattn_ctx* ctx, double* total_ms, int* count, int reset) {
+  if (!ctx || !total_ms || !count) return VATTN_EINVAL;
+  double tot = 0.0;
+  for (size_t i = 0; i < ctx->ev_used; i++) {
+    if (cudaEventSynchronize(ctx->ev_stop[i]) != cudaSuccess) return VATTN_ECUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, ctx->ev_start[i], ctx->ev_stop[i]) != cudaSuccess) return VATTN_ECUDA;
+    tot += ms;
+  }
+  *total_ms = tot;
+  *count = static_cast<int>(ctx->ev_used);
+  if (reset) ctx->ev_used = 0;
+  return VATTN_OK;
+}
+
+int vattn_last_error(vattn_ctx* ctx, int sync) {
+  if (!ctx) return VATTN_EINVAL;
+  if (!sync) return ctx->last_status;
+  if (cudaDeviceSynchronize() != cudaSuccess) return VATTN_ECUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, ctx->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return VATTN_ECUDA;
+  if (cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess) return VATTN_ECUDA;
+  return static_cast<int>(v);
+}
+
+int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* page_table, const int32_t* seq_lens, int batch,
+                 const vattn_params* prm, float* out, int32_t* sel_idx, int32_t* sel_count,
+                 int32_t* budgets, int32_t* head_need, void* stream) {
+  if (!ctx) return VATTN_EINVAL;
+  ctx->last_status = VATTN_EINVAL;
+  const vattn_config& c = ctx->cfg;
+  if (!prm || !q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !sel_idx ||
+      !sel_count || !budgets || !head_need)
+    return VATTN_EINVAL;
+  if (batch < 0 || batch > c.max_batch) return VATTN_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return VATTN_EINVAL;
+  if (prm->sinks < 0 || prm->window < 0 || prm->topk_abs < 0 || prm->topk_den < 0 ||
+      prm->topk_num < 0 || prm->pilot_num < 0 || prm->pilot_den < 0)
+    return VATTN_EINVAL;
+  if (prm->topk_den > 0 && prm->topk_num > prm->topk_den) return VATTN_EINVAL;
+  if (prm->pilot_den > 0 && prm->pilot_num > prm->pilot_den) return VATTN_EINVAL;
+  if (prm->pilot_min < 2 || prm->pilot_min > (1 << 24)) return VATTN_EINVAL;
+  if (!(prm->eps > 0.0f) || !isfinite(prm->eps)) return VATTN_EINVAL;
+  if (!(prm->delta > 0.0f && prm->delta < 1.0f)) return VATTN_EINVAL;
+  if (prm->num_pages < 1) return VATTN_EINVAL;
+  if (c.proxy == VATTN_SPARQ && (!prm->k_t_cache || !aligned16(prm->k_t_cache))) return VATTN_EINVAL;
+  if (c.proxy == VATTN_LOKI && (!prm->k_proj_cache || !prm->proj_basis || !aligned16(prm->k_proj_cache)))
+    return VATTN_EINVAL;
+  Kernels K;
+  if (!pick(c, ctx->G, &K)) return VATTN_EINVAL;
+  if (batch == 0) {
+    ctx->last_launches = 0;
+    return ctx->last_status = VATTN_OK;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  DevParams P;
+  fill_common(ctx, &P, batch);
+  P.sinks = prm->sinks;
+  P.window = prm->window;
+  P.topk_abs = prm->topk_abs;
+  P.topk_num = prm->topk_num;
+  P.topk_den = prm->topk_den;
+  P.pilot_min = prm->pilot_min;
+  P.pilot_num = prm->pilot_num;
+  P.pilot_den = prm->pilot_den;
+  P.eps = prm->eps;
+  if (static_cast<double>(prm->delta) != ctx->cached_delta) {
+    ctx->cached_delta = static_cast<double>(prm->delta);
+    ctx->cached_z = normal_upper_quantile(ctx->cached_delta);
+  }
+  P.z = ctx->cached_z;
+  P.seed = prm->seed;
+  P.num_pages = prm->num_pages;
+  P.q = q;
+  P.k = k_cache;
+  P.v = v_cache;
+  P.kt = prm->k_t_cache;
+  P.kp = prm->k_proj_cache;
+  P.basis = prm->proj_basis;
+  P.page_table = page_table;
+  P.seq_lens = seq_lens;
+  P.out = out;
+  P.sel = sel_idx;
+  P.sel_count = sel_count;
+  P.budgets = budgets;
+  P.head_need = head_need;
+  P.SA = splits_for(ctx->num_sms * 2, P.units);
+  P.SB = splits_for(ctx->num_sms * 2 * ctx->gather_occ, P.units);
+  P.dense = 0;
+  const dim3 seg_grid(P.units, ctx->nseg);
+
+  int launches = 0;
+  K.prep<<<P.units + 1, 128, 0, st>>>(P);
+  launches++;
+  void (*score)(DevParams) = c.proxy == VATTN_SPARQ ? K.score_sparq
+                             : c.proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
+  const bool timed = ctx->timing != 0;
+  if (timed) {
+    if (ctx->ev_used == ctx->ev_start.size()) {
+      cudaEvent_t a, b;
+      cudaEventCreate(&a);
+      cudaEventCreate(&b);
+      ctx->ev_start.push_back(a);
+      ctx->ev_stop.push_back(b);
+    }
+    cudaEventRecord(ctx->ev_start[ctx->ev_used], st);
+  }
+  score<<<ctx->score_grid, 256, 0, st>>>(P);
+  launches++;
+  if (timed) {
+    cudaEventRecord(ctx->ev_stop[ctx->ev_used], st);
+    ctx->ev_used++;
+  }
+  vattn::k_sel_hist<2><<<seg_grid, 256, 0, st>>>(P);
+  vattn::k_sel_hist<3><<<seg_grid, 256, 0, st>>>(P);
+  vattn::k_sel_count<<<seg_grid, 256, 0, st>>>(P);
+  vattn::k_sel_write<<<seg_grid, 256, 0, st>>>(P);
+  launches += 4;
+  K.pilot<<<dim3(P.units, P.SA), 256, 0, st>>>(P);
+  K.budget<<<P.units, 256, 0, st>>>(P);
+  K.gather<<<dim3(P.units, P.SB), 256, 0, st>>>(P);
+  K.combine<<<P.units, ctx->G * c.head_dim, 0, st>>>(P);
+  launches += 4;
+  return finish(ctx, launches);
+}
+
+int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* seq_lens, int batch, int num_pages,
+                       float* out, void* stream) {
+  if (!ctx) return VATTN_EINVAL;
+  ctx->last_status = VATTN_EINVAL;
+  const vattn_config& c = ctx->cfg;
+  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return VATTN_EINVAL;
+  if (batch < 0 || batch > c.max_batch || num_pages < 1) return VATTN_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return VATTN_EINVAL;
+  Kernels K;
+  if (!pick(c, ctx->G, &K)) return VATTN_EINVAL;
+  if (batch == 0) {
+    ctx->last_launches = 0;
+    return ctx->last_status = VATTN_OK;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevParams P;
+  fill_common(ctx, &P, batch);
+  // no selection: sinks cover everything, so every unit is a deterministic
+  // set of all positions with no middle to rank
+  P.sinks = c.max_ctx;
+  P.window = 0;
+  P.pilot_min = 2;
+  P.eps = 1.0f;
+  P.num_pages = num_pages;
+  P.proxy = VATTN_EXACT;
+  P.q = q;
+  P.k = k_cache;
+  P.v = v_cache;
+  P.page_table = page_table;
+  P.seq_lens = seq_lens;
+  P.out = out;
+  P.SB = splits_for(ctx->num_sms * 4 * ctx->gather_occ, P.units);
+  P.dense = 1;
+  // prep only validates and fills the unit state here; its index writes go to
+  // the workspace copy of the selection list, never to caller memory
+  P.sel = reinterpret_cast<int*>(ctx->ordk);
+  K.prep<<<P.units + 1, 128, 0, st>>>(P);
+  K.gather<<<dim3(P.units, P.SB), 256, 0, st>>>(P);
+  K.combine<<<P.units, ctx->G * c.head_dim, 0, st>>>(P);
+  return finish(ctx, 3);
+}
+
+}  // extern "C"

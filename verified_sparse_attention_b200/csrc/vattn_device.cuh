@@ -1,0 +1,328 @@
+// Device-side building blocks of the decode step: element unpacking, the
+// fixed-order fp32 dot, the order-preserving score key, Philox4x32-10, the
+// fixed-order exp used by the budget statistics, and the shared parameter
+// block every kernel receives.
+//
+// Arithmetic that decides an integer (ranking order, sample positions,
+// budgets) is written with explicit round-to-nearest intrinsics so the
+// compiler cannot contract or reorder it; see the comments at each function
+// for the order it fixes.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vattn {
+
+constexpr int kHist1 = 2048;  // bins of digit 1 (key bits 31..21)
+constexpr int kHist2 = 2048;  // bins of digit 2 (key bits 20..10)
+constexpr int kHist3 = 1024;  // bins of digit 3 (key bits 9..0)
+constexpr int kHistAll = kHist1 + kHist2 + kHist3;
+constexpr int kSeg = 4096;         // positions per selection CTA (256 threads x 16)
+constexpr int kTopkSmem = 6144;    // top-k lists up to this length are staged in shared memory
+constexpr int kSbMax = 64;         // partial slots per unit in the gather
+
+// Per-unit (sequence b, KV head h) state written by the prep and budget kernels.
+struct UnitInfo {
+  int n;         // sequence length (0 when the sequence failed validation)
+  int s1;        // end of the sinks: min(sinks, n)
+  int wst;       // start of the window: max(n - window, s1)
+  int k;         // top-k size, capped by the middle's length
+  int p;         // pilot size
+  int ntail;     // tail size: (wst - s1) - k
+  int nI;        // |I_f| = s1 + k + (n - wst)
+  int mode;      // 0: no tail; 1: tail taken whole without a pilot; 2: pilot + budget
+  int bsz;       // final sample size b (ntail when the tail is taken whole)
+  int exhausted; // 1 when the whole tail is taken with weight 1
+  int nitems;    // entries gathered: nI + bsz
+  int pad0;
+  unsigned thr;  // top-k threshold key
+  int need_eq;   // how many keys equal to thr (lowest positions first) are taken
+  int pad1, pad2;
+};
+
+struct DevParams {
+  // shapes
+  int Hq, Hkv, G, D;
+  int pps;        // page-table entries per sequence
+  int ps_log2;    // log2(page_size)
+  int max_ctx, batch, units, num_pages;
+  int proxy, rank;
+  // per-call parameters
+  int sinks, window, topk_abs, topk_num, topk_den, pilot_min, pilot_num, pilot_den;
+  float eps, scale;
+  double z;
+  unsigned long long seed;
+  int nseg, SA, SB, dense;
+  // inputs
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* kt;
+  const void* kp;
+  const float* basis;
+  const int* page_table;
+  const int* seq_lens;
+  // outputs
+  float* out;
+  int* sel;
+  int* sel_count;
+  int* budgets;
+  int* head_need;
+  // workspace
+  UnitInfo* info;
+  float* qbar;      // [units][D]: ranking query (group mean)
+  float* qsel;      // [units][D]: SparQ query values at the chosen dims, or the Loki projected query
+  int* dims;        // [units][D]: SparQ chosen dims, ascending
+  unsigned* ordk;   // [units][max_ctx]: ranking-score keys over the middle
+  unsigned* hist;   // [units][kHistAll]
+  unsigned* segcnt; // [units][nseg][2]
+  float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
+  float* partial;   // [units][kSbMax][G][4 + 2D]: (m_f, l_f, m_s, l_s, acc_f[D], acc_s[D])
+  long long* prefix;// [units + 1]: score-pass work prefix
+  unsigned* err;
+};
+
+// ---------------------------------------------------------------- elements
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int kPer16 = 4;
+  __device__ static __forceinline__ void unpack(const uint4& r, float (&x)[4]) {
+    x[0] = __uint_as_float(r.x);
+    x[1] = __uint_as_float(r.y);
+    x[2] = __uint_as_float(r.z);
+    x[3] = __uint_as_float(r.w);
+  }
+  __device__ static __forceinline__ float load(const void* base, size_t i) {
+    return static_cast<const float*>(base)[i];
+  }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kPer16 = 8;
+  // word w holds element 2w in its low half and 2w+1 in its high half
+  __device__ static __forceinline__ void unpack(const uint4& r, float (&x)[8]) {
+    x[0] = __uint_as_float(r.x << 16);
+    x[1] = __uint_as_float(r.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(r.y << 16);
+    x[3] = __uint_as_float(r.y & 0xFFFF0000u);
+    x[4] = __uint_as_float(r.z << 16);
+    x[5] = __uint_as_float(r.z & 0xFFFF0000u);
+    x[6] = __uint_as_float(r.w << 16);
+    x[7] = __uint_as_float(r.w & 0xFFFF0000u);
+  }
+  __device__ static __forceinline__ float load(const void* base, size_t i) {
+    return __uint_as_float(static_cast<unsigned>(static_cast<const unsigned short*>(base)[i]) << 16);
+  }
+};
+
+// Streaming 16-byte load (cache-streaming: likely accessed once).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  return __ldcs(static_cast<const uint4*>(p));
+}
+
+// Read-only 16-byte load for gathered rows.
+__device__ __forceinline__ uint4 ld_gather(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------- fixed-order dot
+// One 16-byte chunk of the dot: a fused multiply-add chain from 0 over the
+// chunk's elements in ascending order.
+template <typename T>
+__device__ __forceinline__ float chunk_dot(const float* q, const uint4& raw) {
+  constexpr int E = Elem<T>::kPer16;
+  float x[E];
+  Elem<T>::unpack(raw, x);
+  float acc = 0.0f;
+#pragma unroll
+  for (int i = 0; i < E; i++) acc = __fmaf_rn(q[i], x[i], acc);
+  return acc;
+}
+
+// Chunk sums of one row live in the L lanes of an aligned lane group (lane li
+// holds chunk li). The row's dot is the halving-stride tree over chunks:
+// chunk l += chunk l + L/2, then l += l + L/4, ..., l += l + 1. A butterfly
+// with xor offsets L/2, ..., 1 produces exactly these sums in every lane
+// (each stage adds the same two operands, and fp addition is commutative).
+template <int L>
+__device__ __forceinline__ float group_allreduce(float v) {
+#pragma unroll
+  for (int o = L / 2; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
+
+// The same tree for U rows at once (U <= L): at the first log2(U) stages each
+// lane keeps half of its rows and receives its partner's partials for them,
+// so U rows cost (U - 1) + log2(L/U) shuffles instead of U*log2(L). Each stage
+// still adds the partials of lanes x and x^o for a row, so every row's sum is
+// the same tree as group_allreduce. Afterwards the lanes
+// [r*(L/U), (r+1)*(L/U)) of the group hold row r.
+template <int L, int U>
+__device__ __forceinline__ float reduce_rows(float (&a)[U], int li) {
+  constexpr int LOGL = ilog2c(L);
+  constexpr int LOGU = ilog2c(U);
+#pragma unroll
+  for (int s = 0; s < LOGL; s++) {
+    const int o = L >> (s + 1);
+    if (s < LOGU) {
+      const int half = U >> (s + 1);
+      const bool up = (li & o) != 0;
+#pragma unroll
+      for (int i = 0; i < half; i++) {
+        float send = up ? a[i] : a[i + half];
+        float keep = up ? a[i + half] : a[i];
+        a[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, o));
+      }
+    } else {
+      a[0] = __fadd_rn(a[0], __shfl_xor_sync(0xffffffffu, a[0], o));
+    }
+  }
+  return a[0];
+}
+
+template <int L, int U>
+__device__ __forceinline__ int reduce_rows_row(int li) {
+  constexpr int LOGU = ilog2c(U);
+  int r = 0;
+#pragma unroll
+  for (int s = 0; s < LOGU; s++) {
+    const int o = L >> (s + 1);
+    if (li & o) r += U >> (s + 1);
+  }
+  return r;
+}
+
+// ---------------------------------------------------------------- keys
+// Order-preserving map of an fp32 score onto uint32; -0 maps like +0.
+__device__ __forceinline__ unsigned ord_key(float f) {
+  if (f == 0.0f) f = 0.0f;
+  unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------- Philox4x32-10
+// Salmon, Moraes, Dror, Shaw (SC'11). Draw t of unit (b, h) is word t%4 of the
+// block with counter (t/4, b, h, 0) under key (seed low, seed high).
+__device__ __forceinline__ unsigned draw_word(unsigned long long seed, unsigned b, unsigned h,
+                                              unsigned t) {
+  unsigned c0 = t >> 2, c1 = b, c2 = h, c3 = 0u;
+  unsigned k0 = static_cast<unsigned>(seed), k1 = static_cast<unsigned>(seed >> 32);
+#pragma unroll
+  for (int round = 0; round < 10; round++) {
+    if (round > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const unsigned lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const unsigned lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const unsigned n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  const unsigned w = t & 3u;
+  return w == 0 ? c0 : (w == 1 ? c1 : (w == 2 ? c2 : c3));
+}
+
+// Lemire multiply-shift: a 32-bit uniform word onto [0, n).
+__device__ __forceinline__ int lemire(unsigned u, int n) {
+  return static_cast<int>((static_cast<unsigned long long>(u) * static_cast<unsigned>(n)) >> 32);
+}
+
+// ---------------------------------------------------------------- fixed-order exp
+// e^x for x <= 0 in fp32 (Cody-Waite): n = rint(x*log2 e); r = (x - n*C1) - n*C2
+// with ln 2 = C1 + C2, C1 = 0.693359375 (9 significant bits, so n*C1 is exact);
+// e^r by its degree-7 Taylor polynomial in Horner form with fused steps;
+// result p * 2^n. Below -87 the result leaves the normal range and 0 is
+// returned. Used only where the value feeds the integer budget statistics.
+__device__ __forceinline__ float vexp(float x) {
+  if (!(x >= -87.0f)) return 0.0f;
+  const float n = rintf(__fmul_rn(x, 1.44269504088896341f));
+  float r = __fmaf_rn(-n, 0.693359375f, x);
+  r = __fmaf_rn(-n, -2.12194440054690583e-4f, r);
+  float p = 1.98412698412698413e-4f;           // 1/7!
+  p = __fmaf_rn(p, r, 1.38888888888888889e-3f); // 1/6!
+  p = __fmaf_rn(p, r, 8.33333333333333333e-3f); // 1/5!
+  p = __fmaf_rn(p, r, 4.16666666666666667e-2f); // 1/4!
+  p = __fmaf_rn(p, r, 1.66666666666666667e-1f); // 1/3!
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const float scale = __int_as_float((static_cast<int>(n) + 127) << 23);
+  return __fmul_rn(p, scale);
+}
+
+// ---------------------------------------------------------------- block helpers
+// Inclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ unsigned block_inclusive_scan(unsigned v, unsigned* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned w = lane < nw ? s_warp[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      unsigned t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    if (lane < nw) s_warp[lane] = w;
+  }
+  __syncthreads();
+  const unsigned base = warp > 0 ? s_warp[warp - 1] : 0u;
+  __syncthreads();
+  return v + base;
+}
+
+__device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) s_warp[warp] = v;
+  __syncthreads();
+  unsigned tot = 0;
+  for (int i = 0; i < nw; i++) tot += s_warp[i];
+  __syncthreads();
+  return tot;
+}
+
+// Radix-select step over a histogram: find the bin holding the krem-th largest
+// key (counting from the top bin) and the rank left inside that bin.
+// Block of 256 threads; nbins a multiple of 256.
+__device__ __forceinline__ void find_digit(const unsigned* __restrict__ hist, int nbins, int krem,
+                                           int* s_digit, int* s_krem, unsigned* s_warp) {
+  const int per = nbins / blockDim.x;
+  const int t = threadIdx.x;
+  const int hi = nbins - t * per;  // this thread's bins are [hi - per, hi), scanned downwards
+  unsigned sum = 0;
+  for (int i = 1; i <= per; i++) sum += hist[hi - i];
+  const unsigned incl = block_inclusive_scan(sum, s_warp);
+  const unsigned excl = incl - sum;
+  if (excl < static_cast<unsigned>(krem) && static_cast<unsigned>(krem) <= incl) {
+    unsigned c = excl;
+    for (int i = 1; i <= per; i++) {
+      const unsigned hcount = hist[hi - i];
+      if (c + hcount >= static_cast<unsigned>(krem)) {
+        *s_digit = hi - i;
+        *s_krem = krem - static_cast<int>(c);
+        break;
+      }
+      c += hcount;
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace vattn
