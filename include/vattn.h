@@ -43,8 +43,8 @@
  *              0 when there is no tail)
  *   head_need  [batch][Hq] int32: n_h, the CLT size required by query head
  *              hq (N_tail when the tail was taken whole before any pilot)
- * A contiguous cache is one page per sequence: page_size = max_ctx (a power
- * of two) and page_table[b][0] = b.
+ * A contiguous cache is one page per sequence: page_size >= max_ctx (a
+ * multiple of 16) and page_table[b][0] = b.
  *
  * Return codes: VATTN_OK, or a negative VATTN_E* code for bad host arguments
  * (nothing is launched) or a CUDA launch failure. Device-side violations (a
@@ -84,7 +84,8 @@ typedef struct {
   int num_kv_heads; /* Hkv >= 1                                                  */
   int head_dim;     /* d in {64, 128}                                            */
   int dtype;        /* VATTN_FP32 or VATTN_BF16, for q and every cache          */
-  int page_size;    /* power of two >= 16 (contiguous cache: = max_ctx)          */
+  int page_size;    /* rows per page, a multiple of 16 (contiguous cache: max_ctx */
+                    /* rounded up to a multiple of 16)                            */
   int max_batch;    /* upper bound on `batch` in every call                      */
   int max_ctx;      /* upper bound on seq_lens[b]; 1 <= max_ctx <= 2^24          */
   int proxy;        /* VATTN_EXACT, VATTN_SPARQ or VATTN_LOKI                    */

@@ -64,12 +64,6 @@ double normal_upper_quantile(double delta) {
   return 0.5 * (lo + hi);
 }
 
-bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
-int log2i(int x) {
-  int r = 0;
-  while ((1 << r) < x) r++;
-  return r;
-}
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -128,7 +122,7 @@ int check_config(const vattn_config* c) {
   if (!(G == 1 || G == 2 || G == 4 || G == 8)) return VATTN_EINVAL;
   if (!(c->head_dim == 64 || c->head_dim == 128)) return VATTN_EINVAL;
   if (!(c->dtype == VATTN_FP32 || c->dtype == VATTN_BF16)) return VATTN_EINVAL;
-  if (!is_pow2(c->page_size) || c->page_size < 16) return VATTN_EINVAL;
+  if (c->page_size < 16 || c->page_size % 16) return VATTN_EINVAL;
   if (c->max_batch < 1 || c->max_ctx < 1 || c->max_ctx > (1 << 24)) return VATTN_EINVAL;
   if (c->proxy == VATTN_SPARQ) {
     if (c->proxy_rank < 1 || c->proxy_rank > c->head_dim) return VATTN_EINVAL;
@@ -148,7 +142,8 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->G = ctx->G;
   P->D = c.head_dim;
   P->pps = (c.max_ctx + c.page_size - 1) / c.page_size;
-  P->ps_log2 = log2i(c.page_size);
+  P->ps = c.page_size;
+  P->ps_magic = ~0ull / static_cast<unsigned long long>(c.page_size) + 1ull;
   P->max_ctx = c.max_ctx;
   P->batch = batch;
   P->units = batch * c.num_kv_heads;

@@ -46,7 +46,8 @@ struct DevParams {
   // shapes
   int Hq, Hkv, G, D;
   int pps;        // page-table entries per sequence
-  int ps_log2;    // log2(page_size)
+  int ps;         // page size (rows per page)
+  unsigned long long ps_magic;  // ceil(2^64 / ps): j / ps = mulhi(j, ps_magic) for j < 2^24
   int max_ctx, batch, units, num_pages;
   int proxy, rank;
   // per-call parameters

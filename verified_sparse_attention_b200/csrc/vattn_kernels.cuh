@@ -26,14 +26,17 @@ namespace vattn {
 
 constexpr int kProxyExact = 0, kProxySparq = 1, kProxyLoki = 2;
 
-__device__ __forceinline__ int page_of(const DevParams& P, int b, int j) {
-  return P.page_table[static_cast<size_t>(b) * P.pps + (j >> P.ps_log2)];
+// Page-table slot of position j (exact for 0 <= j < 2^24, page size >= 2).
+__device__ __forceinline__ int page_slot(const DevParams& P, int j) {
+  return static_cast<int>(__umul64hi(static_cast<unsigned long long>(j), P.ps_magic));
 }
 
 // Element offset of row j of unit (b, h) in a [pages][Hkv][page_size][W] cache.
 __device__ __forceinline__ size_t row_off(const DevParams& P, int b, int h, int j, int W) {
-  const size_t page = static_cast<size_t>(page_of(P, b, j));
-  return ((page * P.Hkv + h) << P.ps_log2 | static_cast<size_t>(j & ((1 << P.ps_log2) - 1))) * W;
+  const int slot = page_slot(P, j);
+  const size_t page = static_cast<size_t>(P.page_table[static_cast<size_t>(b) * P.pps + slot]);
+  const int row = j - slot * P.ps;
+  return ((page * P.Hkv + h) * P.ps + row) * static_cast<size_t>(W);
 }
 
 // Regions of a sequence of length n (sinks [0,s1), middle [s1,wst), window [wst,n)).
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   int n = P.seq_lens[b];
   const bool bad_len = n < 0 || n > P.max_ctx;
   if (bad_len) n = 0;
-  const int npages = (n + (1 << P.ps_log2) - 1) >> P.ps_log2;
+  const int npages = (n + P.ps - 1) / P.ps;
   int bad = 0;
   for (int i = tid; i < npages; i += blockDim.x) {
     const int pid = P.page_table[static_cast<size_t>(b) * P.pps + i];
@@ -303,7 +306,6 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
   const long long end = total * (blockIdx.x + 1) / gridDim.x;
   if (beg >= end) return;
   const int r = P.rank;
-  const int psm = (1 << P.ps_log2) - 1;
   int u = find_unit(P.prefix, P.units, beg);
   long long cur = beg;
   while (cur < end) {
@@ -324,9 +326,11 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
       unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
       for (long long gi = gb + threadIdx.x; gi < ge; gi += blockDim.x) {
         const int j0 = static_cast<int>(gi) * V;
-        const size_t page = static_cast<size_t>(page_of(P, b, j0));
-        const size_t rowbase = ((page * P.Hkv + h) * D) << P.ps_log2;
-        const int off = j0 & psm;
+        const int slot = page_slot(P, j0);
+        const size_t page = static_cast<size_t>(P.page_table[static_cast<size_t>(b) * P.pps + slot]);
+        const size_t ps = static_cast<size_t>(P.ps);
+        const size_t rowbase = (page * P.Hkv + h) * D * ps;
+        const int off = j0 - slot * P.ps;
         float acc[V];
 #pragma unroll
         for (int v = 0; v < V; v++) acc[v] = 0.0f;
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
           uint4 raw[8];
 #pragma unroll
           for (int c = 0; c < 8; c++)
-            raw[c] = ld_stream(kt + rowbase + (static_cast<size_t>(s_dim[t + c]) << P.ps_log2) + off);
+            raw[c] = ld_stream(kt + rowbase + static_cast<size_t>(s_dim[t + c]) * ps + off);
 #pragma unroll
           for (int c = 0; c < 8; c++) {
             float x[V];
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
           }
         }
         for (; t < r; t++) {
-          const uint4 raw = ld_stream(kt + rowbase + (static_cast<size_t>(s_dim[t]) << P.ps_log2) + off);
+          const uint4 raw = ld_stream(kt + rowbase + static_cast<size_t>(s_dim[t]) * ps + off);
           float x[V];
           Elem<T>::unpack(raw, x);
           const float qv = s_qv[t];
@@ -586,11 +590,12 @@ __global__ void __launch_bounds__(256) k_pilot(DevParams P) {
   const T* kc = static_cast<const T*>(P.k);
   float* ps = P.pscore + static_cast<size_t>(u) * P.max_ctx * G;
   constexpr int UU = 2;
-  for (int i0 = ib + (warp * RPW + grp) * UU; i0 < ie; i0 += nwarps * RPW * UU) {
+  // warp-uniform trip count: every lane runs the shuffles of group_allreduce
+  for (int wb = ib + warp * RPW * UU; wb < ie; wb += nwarps * RPW * UU) {
     uint4 raw[UU];
 #pragma unroll
     for (int k = 0; k < UU; k++) {
-      const int i = i0 + k;
+      const int i = wb + k * RPW + grp;
       if (i < ie) {
         const int j = item_position(P, u, inf, topk, i, false);
         raw[k] = ld_gather(kc + row_off(P, b, h, j, D) + li * E);
@@ -600,7 +605,7 @@ __global__ void __launch_bounds__(256) k_pilot(DevParams P) {
     }
 #pragma unroll
     for (int k = 0; k < UU; k++) {
-      const int i = i0 + k;
+      const int i = wb + k * RPW + grp;
 #pragma unroll
       for (int g = 0; g < G; g++) {
         const float s = __fmul_rn(group_allreduce<L>(chunk_dot<T>(q[g], raw[k])), P.scale);
@@ -803,12 +808,13 @@ __global__ void __launch_bounds__(256) k_gather(DevParams P) {
 #pragma unroll
       for (int e = 0; e < E; e++) acc[g][e] = 0.0f;
     }
-    for (int i0 = rb + gid * UU; i0 < re; i0 += NGRP * UU) {
+    // warp-uniform trip count: every lane runs the shuffles of group_allreduce
+    for (int wb = rb + warp * RPW * UU; wb < re; wb += NGRP * UU) {
       uint4 kr[UU], vr[UU];
       bool ok[UU];
 #pragma unroll
       for (int k = 0; k < UU; k++) {
-        const int i = i0 + k;
+        const int i = wb + k * RPW + grp;
         ok[k] = i < re;
         if (ok[k]) {
           int j = i;

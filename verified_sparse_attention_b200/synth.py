@@ -93,10 +93,11 @@ PAGED_EPS_SWEEP = (0.01, 0.05, 0.1, 0.2)
 
 
 def scaled(w, *, max_ctx, min_ctx=None, batch=None, page_size=None, **kw):
-    """Same recipe at a smaller size (page size shrinks with a contiguous cache)."""
+    """Same recipe at a smaller size (a contiguous cache keeps one page per sequence,
+    its size max_ctx rounded up to a multiple of 16)."""
     min_ctx = max_ctx if min_ctx is None else min_ctx
     if page_size is None:
-        page_size = max_ctx if w.page_size == w.max_ctx else w.page_size
+        page_size = -(-max_ctx // 16) * 16 if w.page_size >= w.max_ctx else w.page_size
     return w.replace(max_ctx=max_ctx, min_ctx=min_ctx, page_size=page_size,
                      batch=w.batch if batch is None else batch, **kw)
 
