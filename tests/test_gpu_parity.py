@@ -114,6 +114,17 @@ def test_dtype_and_head_dim(dtype, d):
     check(w)
 
 
+def test_long_max_ctx_uses_grid_wide_selection():
+    # a context bound whose per-CTA key segment does not fit in shared memory
+    # selects the top-k with the grid-wide passes instead of one cluster per unit
+    small = synth.scaled(W["gqa_32k"], max_ctx=9000, batch=1, num_q_heads=8, num_kv_heads=2)
+    cpu = synth.make_inputs(small)
+    w = small.replace(max_ctx=600000, min_ctx=600000)      # same page size, longer bound
+    pad = torch.full((1, w.pages_per_seq - cpu["page_table"].shape[1]), -1, dtype=torch.int32)
+    cpu["page_table"] = torch.cat([cpu["page_table"], pad], 1)
+    check(w, inputs=cpu)
+
+
 def test_no_topk_and_large_topk():
     base = synth.scaled(W["tiny_f32"], max_ctx=2000)
     check(base.replace(topk_abs=0))

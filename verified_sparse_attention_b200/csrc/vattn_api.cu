@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "vattn.h"
@@ -21,7 +22,14 @@ struct vattn_ctx {
   int units_max = 0;
   int nseg = 0;
   int score_grid = 0;
-  int gather_occ = 1;
+  int CD = 0, CS = 0;      // gather grid sizes (det/dense, sample)
+  size_t gather_smem = 0;   // det/dense gather
+  size_t sample_smem = 0;   // sample gather (adds its slice prefix)
+  size_t budget_smem = 0;
+  size_t combine_smem = 0;
+  int combine_scr = 0;      // floats
+  size_t select_smem = 0;   // 0: the selection runs as four grid-wide passes
+  int draw_splits = 1;
   size_t ws_bytes = 0;
   void* ws = nullptr;
   // carved workspace
@@ -33,8 +41,13 @@ struct vattn_ctx {
   unsigned* hist = nullptr;
   unsigned* segcnt = nullptr;
   float* pscore = nullptr;
-  float* partial = nullptr;
   long long* prefix = nullptr;
+  unsigned* cnt = nullptr;
+  unsigned* gcnt = nullptr;
+  long long* pre_det = nullptr;
+  long long* pre_samp = nullptr;
+  float* rec_det = nullptr;
+  float* rec_samp = nullptr;
   unsigned* err = nullptr;
   // state
   int last_status = VATTN_OK;
@@ -73,10 +86,13 @@ struct Kernels {
   void (*score_exact)(DevParams);
   void (*score_loki)(DevParams);
   void (*score_sparq)(DevParams);
-  void (*pilot)(DevParams);
+  void (*det)(DevParams);
+  void (*sample)(DevParams);
+  void (*dense)(DevParams);
   void (*budget)(DevParams);
-  void (*gather)(DevParams);
-  void (*combine)(DevParams);
+  void (*combine_sample)(DevParams);
+  void (*combine_dense)(DevParams);
+  size_t gather_smem;
 };
 
 template <typename T, int D, int G>
@@ -86,10 +102,13 @@ Kernels kernels_for() {
   k.score_exact = vattn::k_score_rows<T, D>;
   k.score_loki = vattn::k_score_rows<T, 32>;
   k.score_sparq = vattn::k_score_sparq<T, D>;
-  k.pilot = vattn::k_pilot<T, D, G>;
-  k.budget = vattn::k_budget<G>;
-  k.gather = vattn::k_gather<T, D, G>;
-  k.combine = vattn::k_combine<D, G>;
+  k.det = vattn::k_gather<T, D, G, vattn::kModeDet>;
+  k.sample = vattn::k_gather<T, D, G, vattn::kModeSample>;
+  k.dense = vattn::k_gather<T, D, G, vattn::kModeDense>;
+  k.budget = vattn::k_budget<D, G>;
+  k.combine_sample = vattn::k_combine<D, G, vattn::kModeSample>;
+  k.combine_dense = vattn::k_combine<D, G, vattn::kModeDense>;
+  k.gather_smem = vattn::GatherShape<T, D, G>::SMEM;
   return k;
 }
 
@@ -159,16 +178,36 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->hist = ctx->hist;
   P->segcnt = ctx->segcnt;
   P->pscore = ctx->pscore;
-  P->partial = ctx->partial;
   P->prefix = ctx->prefix;
+  P->cnt = ctx->cnt;
+  P->gcnt = ctx->gcnt;
+  P->pre_det = ctx->pre_det;
+  P->pre_samp = ctx->pre_samp;
+  P->rec_det = ctx->rec_det;
+  P->rec_samp = ctx->rec_samp;
+  P->CD = ctx->CD;
+  P->CS = ctx->CS;
+  P->combine_scr = ctx->combine_scr;
   P->err = ctx->err;
 }
 
-int splits_for(int want, int units) {
-  int s = (want + units - 1) / units;
-  if (s < 1) s = 1;
-  if (s > vattn::kSbMax) s = vattn::kSbMax;
-  return s;
+// Launch with programmatic dependent launch: the kernel may be scheduled while
+// its predecessor on the stream drains; it waits (griddepcontrol.wait) before
+// reading the predecessor's results.
+void launch(void (*kern)(DevParams), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const DevParams& P,
+            int* count) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, P);
+  (*count)++;
 }
 
 int finish(vattn_ctx* ctx, int launches) {
@@ -213,16 +252,53 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const size_t U = static_cast<size_t>(cfg->max_batch) * cfg->num_kv_heads;
   ctx->units_max = static_cast<int>(U);
   ctx->nseg = (cfg->max_ctx + vattn::kSeg - 1) / vattn::kSeg;
+
+  // grid sizes: the score pass and the gathers run one wave of resident CTAs
+  void (*score)(DevParams) = cfg->proxy == VATTN_SPARQ ? K.score_sparq
+                             : cfg->proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
+  ctx->score_grid = (occ < 1 ? 1 : occ) * ctx->num_sms;
+  ctx->gather_smem = K.gather_smem;
+  ctx->sample_smem = K.gather_smem + (2 * U + 1) * sizeof(long long);
+  for (auto fn : {K.det, K.dense})
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->gather_smem));
+  cudaFuncSetAttribute(K.sample, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->sample_smem));
+  int gocc = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, 256, ctx->sample_smem);
+  if (gocc < 1) gocc = 1;
+  ctx->CD = ctx->CS = gocc * ctx->num_sms;
+  // the combine stages (m, l) and a scale factor per (record, head), and a
+  // unit has at most CD + CS + 2 records; the budget stages record maxima
+  ctx->combine_scr = (3 * G + 2) * (ctx->CD + ctx->CS + 2) + 4 * G;
+  ctx->combine_smem = static_cast<size_t>(ctx->combine_scr) * sizeof(float);
+  ctx->budget_smem = std::max(static_cast<size_t>(ctx->CD + 2) * G * sizeof(float),
+                              static_cast<size_t>(vattn::kTopkSmem) * sizeof(int));
+  ctx->draw_splits = std::max(1, (2 * ctx->num_sms + static_cast<int>(U) - 1) / static_cast<int>(U));
+  for (auto fn : {K.combine_sample, K.combine_dense})
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->combine_smem));
+  cudaFuncSetAttribute(K.budget, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->budget_smem));
+  if (cudaGetLastError() != cudaSuccess) {
+    delete ctx;
+    return VATTN_ECUDA;
+  }
+
+  const size_t REC = static_cast<size_t>(G) * (2 + D);
   const size_t sz_info = align256(U * sizeof(UnitInfo));
   const size_t sz_vec = align256(U * D * sizeof(float));
   const size_t sz_ordk = align256(U * cfg->max_ctx * sizeof(unsigned));
   const size_t sz_hist = align256(U * vattn::kHistAll * sizeof(unsigned));
   const size_t sz_seg = align256(U * ctx->nseg * 2 * sizeof(unsigned));
   const size_t sz_ps = align256(U * cfg->max_ctx * G * sizeof(float));
-  const size_t sz_part = align256(U * vattn::kSbMax * G * (4 + 2 * D) * sizeof(float));
   const size_t sz_pre = align256((U + 1) * sizeof(long long));
+  const size_t sz_cnt = align256(U * 2 * sizeof(unsigned));
+  const size_t sz_gcnt = 256;
+  const size_t sz_spre = align256((2 * U + 1) * sizeof(long long));
+  const size_t sz_rdet = align256((ctx->CD + 2 * U) * REC * sizeof(float));
+  const size_t sz_rsmp = align256((ctx->CS + 2 * U) * REC * sizeof(float));
   const size_t sz_err = 256;
-  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_part + sz_pre + sz_err;
+  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_pre + sz_cnt + sz_gcnt +
+                  2 * sz_spre + sz_rdet + sz_rsmp + sz_err;
   if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
     delete ctx;
@@ -237,27 +313,31 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->hist = reinterpret_cast<unsigned*>(p); p += sz_hist;
   ctx->segcnt = reinterpret_cast<unsigned*>(p); p += sz_seg;
   ctx->pscore = reinterpret_cast<float*>(p); p += sz_ps;
-  ctx->partial = reinterpret_cast<float*>(p); p += sz_part;
   ctx->prefix = reinterpret_cast<long long*>(p); p += sz_pre;
+  ctx->cnt = reinterpret_cast<unsigned*>(p); p += sz_cnt;
+  ctx->gcnt = reinterpret_cast<unsigned*>(p); p += sz_gcnt;
+  ctx->pre_det = reinterpret_cast<long long*>(p); p += sz_spre;
+  ctx->pre_samp = reinterpret_cast<long long*>(p); p += sz_spre;
+  ctx->rec_det = reinterpret_cast<float*>(p); p += sz_rdet;
+  ctx->rec_samp = reinterpret_cast<float*>(p); p += sz_rsmp;
   ctx->err = reinterpret_cast<unsigned*>(p);
-  if (cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess) {
+  if (cudaMemset(ctx->ws, 0, ctx->ws_bytes) != cudaSuccess) {
     cudaFree(ctx->ws);
     delete ctx;
     return VATTN_ECUDA;
   }
-  void (*score)(DevParams) = cfg->proxy == VATTN_SPARQ ? K.score_sparq
-                             : cfg->proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
-  int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
-  if (occ < 1) occ = 1;
-  ctx->score_grid = occ * ctx->num_sms;
-  int gocc = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.gather, 256, 0);
-  ctx->gather_occ = gocc < 1 ? 1 : gocc;
-  if (cudaGetLastError() != cudaSuccess) {
-    cudaFree(ctx->ws);
-    delete ctx;
-    return VATTN_ECUDA;
+  // one cluster per unit selects the top-k when each CTA's key segment fits in
+  // shared memory; otherwise the four grid-wide passes do
+  {
+    const size_t seg = (static_cast<size_t>(cfg->max_ctx) + vattn::kSelCluster - 1) / vattn::kSelCluster;
+    const size_t bytes = vattn::kSelFixedSmem + seg * sizeof(unsigned);
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device);
+    if (bytes + 1024 <= static_cast<size_t>(optin) &&
+        cudaFuncSetAttribute(vattn::k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes)) == cudaSuccess)
+      ctx->select_smem = bytes;
+    cudaGetLastError();
   }
   *out = ctx;
   return VATTN_OK;
@@ -369,14 +449,11 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.sel_count = sel_count;
   P.budgets = budgets;
   P.head_need = head_need;
-  P.SA = splits_for(ctx->num_sms * 2, P.units);
-  P.SB = splits_for(ctx->num_sms * 2 * ctx->gather_occ, P.units);
   P.dense = 0;
   const dim3 seg_grid(P.units, ctx->nseg);
 
   int launches = 0;
-  K.prep<<<P.units + 1, 128, 0, st>>>(P);
-  launches++;
+  launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
   void (*score)(DevParams) = c.proxy == VATTN_SPARQ ? K.score_sparq
                              : c.proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
   const bool timed = ctx->timing != 0;
@@ -390,22 +467,25 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     }
     cudaEventRecord(ctx->ev_start[ctx->ev_used], st);
   }
-  score<<<ctx->score_grid, 256, 0, st>>>(P);
-  launches++;
+  launch(score, dim3(ctx->score_grid), dim3(256), 0, st, P, &launches);
   if (timed) {
     cudaEventRecord(ctx->ev_stop[ctx->ev_used], st);
     ctx->ev_used++;
   }
-  vattn::k_sel_hist<2><<<seg_grid, 256, 0, st>>>(P);
-  vattn::k_sel_hist<3><<<seg_grid, 256, 0, st>>>(P);
-  vattn::k_sel_count<<<seg_grid, 256, 0, st>>>(P);
-  vattn::k_sel_write<<<seg_grid, 256, 0, st>>>(P);
-  launches += 4;
-  K.pilot<<<dim3(P.units, P.SA), 256, 0, st>>>(P);
-  K.budget<<<P.units, 256, 0, st>>>(P);
-  K.gather<<<dim3(P.units, P.SB), 256, 0, st>>>(P);
-  K.combine<<<P.units, ctx->G * c.head_dim, 0, st>>>(P);
-  launches += 4;
+  if (ctx->select_smem) {
+    launch(vattn::k_select, dim3(P.units * vattn::kSelCluster), dim3(256), ctx->select_smem, st, P, &launches);
+  } else {
+    launch(vattn::k_sel_hist<2>, seg_grid, dim3(256), 0, st, P, &launches);
+    launch(vattn::k_sel_hist<3>, seg_grid, dim3(256), 0, st, P, &launches);
+    launch(vattn::k_sel_count, seg_grid, dim3(256), 0, st, P, &launches);
+    launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
+  }
+  launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
+  launch(K.det, dim3(ctx->CD), dim3(256), ctx->gather_smem, st, P, &launches);
+  launch(K.budget, dim3(P.units), dim3(256), ctx->budget_smem, st, P, &launches);
+  launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(256), 0, st, P, &launches);
+  launch(K.sample, dim3(ctx->CS), dim3(256), ctx->sample_smem, st, P, &launches);
+  launch(K.combine_sample, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
   return finish(ctx, launches);
 }
 
@@ -441,15 +521,15 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.page_table = page_table;
   P.seq_lens = seq_lens;
   P.out = out;
-  P.SB = splits_for(ctx->num_sms * 4 * ctx->gather_occ, P.units);
   P.dense = 1;
   // prep only validates and fills the unit state here; its index writes go to
   // the workspace copy of the selection list, never to caller memory
   P.sel = reinterpret_cast<int*>(ctx->ordk);
-  K.prep<<<P.units + 1, 128, 0, st>>>(P);
-  K.gather<<<dim3(P.units, P.SB), 256, 0, st>>>(P);
-  K.combine<<<P.units, ctx->G * c.head_dim, 0, st>>>(P);
-  return finish(ctx, 3);
+  int launches = 0;
+  launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
+  launch(K.dense, dim3(ctx->CD), dim3(256), ctx->gather_smem, st, P, &launches);
+  launch(K.combine_dense, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
+  return finish(ctx, launches);
 }
 
 }  // extern "C"

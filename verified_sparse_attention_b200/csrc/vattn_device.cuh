@@ -21,7 +21,6 @@ constexpr int kHist3 = 1024;  // bins of digit 3 (key bits 9..0)
 constexpr int kHistAll = kHist1 + kHist2 + kHist3;
 constexpr int kSeg = 4096;         // positions per selection CTA (256 threads x 16)
 constexpr int kTopkSmem = 6144;    // top-k lists up to this length are staged in shared memory
-constexpr int kSbMax = 64;         // partial slots per unit in the gather
 
 // Per-unit (sequence b, KV head h) state written by the prep and budget kernels.
 struct UnitInfo {
@@ -55,7 +54,9 @@ struct DevParams {
   float eps, scale;
   double z;
   unsigned long long seed;
-  int nseg, SA, SB, dense;
+  int nseg, dense;
+  int CD, CS;       // grid sizes of the det (and dense) and sample gathers
+  int combine_scr;  // floats of shared scratch in k_combine
   // inputs
   const void* q;
   const void* k;
@@ -80,8 +81,13 @@ struct DevParams {
   unsigned* hist;   // [units][kHistAll]
   unsigned* segcnt; // [units][nseg][2]
   float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
-  float* partial;   // [units][kSbMax][G][4 + 2D]: (m_f, l_f, m_s, l_s, acc_f[D], acc_s[D])
   long long* prefix;// [units + 1]: score-pass work prefix
+  unsigned* cnt;    // [units][2]: finished-segment counters of the det and sample gathers
+  unsigned* gcnt;   // finished-CTA counter of the det gather
+  long long* pre_det;   // [2 units + 1]: slice prefix of the det (or dense) gather
+  long long* pre_samp;  // [2 units + 1]: slice prefix of the sample gather
+  float* rec_det;   // [CD + 2 units][G][2 + D]: det (or dense) gather records
+  float* rec_samp;  // [CS + 2 units][G][2 + D]: sample gather records
   unsigned* err;
 };
 
@@ -301,26 +307,40 @@ __device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* s_warp) {
 
 // Radix-select step over a histogram: find the bin holding the krem-th largest
 // key (counting from the top bin) and the rank left inside that bin.
-// Block of 256 threads; nbins a multiple of 256.
-__device__ __forceinline__ void find_digit(const unsigned* __restrict__ hist, int nbins, int krem,
+// Block of 256 threads; NB a multiple of 1024 (each thread reads NB/256 bins
+// with 16-byte loads, all issued before use).
+template <int NB>
+__device__ __forceinline__ void find_digit(const unsigned* __restrict__ hist, int krem,
                                            int* s_digit, int* s_krem, unsigned* s_warp) {
-  const int per = nbins / blockDim.x;
+  constexpr int PER = NB / 256;
+  static_assert(PER % 4 == 0, "bins per thread must fill 16-byte loads");
   const int t = threadIdx.x;
-  const int hi = nbins - t * per;  // this thread's bins are [hi - per, hi), scanned downwards
+  const int lo = NB - (t + 1) * PER;  // this thread's bins are [lo, lo + PER), scanned downwards
+  unsigned v[PER];
+#pragma unroll
+  for (int i = 0; i < PER / 4; i++) {
+    const uint4 w = *reinterpret_cast<const uint4*>(hist + lo + 4 * i);
+    v[4 * i] = w.x;
+    v[4 * i + 1] = w.y;
+    v[4 * i + 2] = w.z;
+    v[4 * i + 3] = w.w;
+  }
   unsigned sum = 0;
-  for (int i = 1; i <= per; i++) sum += hist[hi - i];
+#pragma unroll
+  for (int i = 0; i < PER; i++) sum += v[i];
   const unsigned incl = block_inclusive_scan(sum, s_warp);
   const unsigned excl = incl - sum;
   if (excl < static_cast<unsigned>(krem) && static_cast<unsigned>(krem) <= incl) {
     unsigned c = excl;
-    for (int i = 1; i <= per; i++) {
-      const unsigned hcount = hist[hi - i];
-      if (c + hcount >= static_cast<unsigned>(krem)) {
-        *s_digit = hi - i;
+    bool done = false;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; i--) {
+      if (!done && c + v[i] >= static_cast<unsigned>(krem)) {
+        *s_digit = lo + i;
         *s_krem = krem - static_cast<int>(c);
-        break;
+        done = true;
       }
-      c += hcount;
+      c += v[i];
     }
   }
   __syncthreads();

@@ -10,15 +10,19 @@
 //   k_sel_hist    radix-select digits 2 and 3 (key bits 20..10, 9..0)
 //   k_sel_count   exact threshold; counts above / equal per segment
 //   k_sel_write   ordered compaction of the top-k positions (ascending)
-//   k_pilot       true scores of I_f and the pilot draws (all query heads)
-//   k_budget      per-head CLT budgets from fixed-point statistics
-//   k_gather      split-K softmax-and-accumulate over I_f and the sample
-//   k_combine     merge splits, reweight the sample by N_tail / b, write out
+//   k_gather<det>    gather + softmax-accumulate of I_f and the pilot draws
+//                    (true scores of every query head kept); the unit's last
+//                    CTA computes the per-head CLT budgets
+//   k_gather<sample> the remaining draws (or the whole tail); the unit's last
+//                    CTA merges its records, reweights the sample by N_tail / b
+//                    and writes out (k_gather<dense>: all positions)
 //
 // A unit is one (sequence b, KV head h); u = b * Hkv + h. The method follows
 // "vAttention: A New Approach to Sparse Attention with Guaranteed Accuracy",
 // section "How vAttention Works" and the paragraph after it.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "vattn_device.cuh"
 
@@ -69,6 +73,16 @@ __device__ __forceinline__ long long score_work(const DevParams& P, int n, int V
   return (r.wst + V - 1) / V - r.s1 / V;
 }
 
+// ---------------------------------------------------------------- launch chaining
+// Every kernel is launched with programmatic dependent launch: it may start
+// while its predecessor finishes, and waits here before touching anything the
+// predecessor wrote (no-op when launched without the attribute).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the successor launch once every CTA of this grid has passed this point.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ============================================================ k_prep
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(128) k_prep(DevParams P) {
@@ -78,6 +92,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   __shared__ unsigned s_tot;
   const int tid = threadIdx.x;
   const int u = blockIdx.x;
+  grid_dependency_wait();  // the previous call's kernels still read this workspace
 
   if (u == P.units) {
     // work prefix over units for the persistent score pass
@@ -100,6 +115,40 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
       __syncthreads();
     }
     if (tid == 0) P.prefix[P.units] = carry;
+    // slice prefix of the det (or dense) gather, from the length-checked n; a
+    // sequence whose pages fail validation keeps its items here and is
+    // skipped by the gather, which reads the validated unit state
+    carry = 0;
+    const int ns = 2 * P.units;
+    for (int base = 0; base < ns; base += blockDim.x) {
+      const int sidx = base + tid;
+      unsigned cnt = 0;
+      if (sidx < ns) {
+        int n = P.seq_lens[(sidx >> 1) / P.Hkv];
+        if (n < 0 || n > P.max_ctx) n = 0;
+        if (P.dense) {
+          cnt = (sidx & 1) ? 0u : static_cast<unsigned>(n);
+        } else {
+          const Regions r = regions(P, n);
+          const int ntail = (r.wst - r.s1) - r.k;
+          const int nI = r.s1 + r.k + (n - r.wst);
+          const int mode = ntail == 0 ? 0 : (ntail <= r.p ? 1 : 2);
+          const int n_extra = mode == 2 ? r.p : (mode == 1 ? ntail : 0);
+          const int n_det = mode == 2 ? nI : nI + n_extra;
+          cnt = static_cast<unsigned>((sidx & 1) ? nI + n_extra - n_det : n_det);
+        }
+      }
+      const unsigned incl = block_inclusive_scan(cnt, s_warp);
+      if (sidx < ns) P.pre_det[sidx] = carry + (incl - cnt);
+      if (tid == blockDim.x - 1) s_tot = incl;
+      __syncthreads();
+      carry += s_tot;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      P.pre_det[ns] = carry;
+      P.gcnt[0] = 0u;
+    }
     return;
   }
 
@@ -191,6 +240,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
 
   unsigned* hist = P.hist + static_cast<size_t>(u) * kHistAll;
   for (int i = tid; i < kHistAll; i += blockDim.x) hist[i] = 0u;
+  if (tid < 2) P.cnt[2 * u + tid] = 0u;
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
   for (int i = tid; i < r.s1; i += blockDim.x) sel[i] = i;
   for (int i = tid; i < n - r.wst; i += blockDim.x) sel[r.s1 + r.k + i] = r.wst + i;
@@ -234,6 +284,7 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int grp = lane / L, li = lane % L;
+  grid_dependency_wait();
   const bool loki = P.proxy == kProxyLoki;
   const void* cache = loki ? P.kp : P.k;
   const float* qsrc = loki ? P.qsel : P.qbar;
@@ -299,6 +350,7 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
   __shared__ float s_qv[D];
   __shared__ int s_dim[D];
 
+  grid_dependency_wait();
   for (int i = threadIdx.x; i < kHist1; i += blockDim.x) s_hist[i] = 0u;
   __syncthreads();
   const long long total = P.prefix[P.units];
@@ -388,18 +440,18 @@ __device__ __forceinline__ SelState resolve_digits(const DevParams& P, int u, in
   SelState st{0, 0, 0, k};
   if (threadIdx.x == 0) { s_digit = 0; s_krem = k; }
   __syncthreads();
-  find_digit(hist, kHist1, st.krem, &s_digit, &s_krem, s_warp);
+  find_digit<kHist1>(hist, st.krem, &s_digit, &s_krem, s_warp);
   st.d1 = s_digit;
   st.krem = s_krem;
   __syncthreads();
   if (DEPTH >= 2) {
-    find_digit(hist + kHist1, kHist2, st.krem, &s_digit, &s_krem, s_warp);
+    find_digit<kHist2>(hist + kHist1, st.krem, &s_digit, &s_krem, s_warp);
     st.d2 = s_digit;
     st.krem = s_krem;
     __syncthreads();
   }
   if (DEPTH >= 3) {
-    find_digit(hist + kHist1 + kHist2, kHist3, st.krem, &s_digit, &s_krem, s_warp);
+    find_digit<kHist3>(hist + kHist1 + kHist2, st.krem, &s_digit, &s_krem, s_warp);
     st.d3 = s_digit;
     st.krem = s_krem;
     __syncthreads();
@@ -412,6 +464,7 @@ template <int PASS>
 __global__ void __launch_bounds__(256) k_sel_hist(DevParams P) {
   __shared__ unsigned s_h[kHist2];
   const int u = blockIdx.x, seg = blockIdx.y;
+  grid_dependency_wait();
   const UnitInfo inf = P.info[u];
   if (inf.k <= 0) return;
   const int pb = inf.s1 + seg * kSeg;
@@ -424,8 +477,18 @@ __global__ void __launch_bounds__(256) k_sel_hist(DevParams P) {
   const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
   const unsigned pre = PASS == 2 ? static_cast<unsigned>(st.d1)
                                  : (static_cast<unsigned>(st.d1) << 11 | static_cast<unsigned>(st.d2));
-  for (int j = pb + threadIdx.x; j < pe; j += blockDim.x) {
-    const unsigned o = ordk[j];
+  constexpr int PER = kSeg / 256;
+  unsigned keys[PER];
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    const int j = pb + threadIdx.x + 256 * i;
+    keys[i] = j < pe ? ordk[j] : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    const int j = pb + threadIdx.x + 256 * i;
+    const unsigned o = keys[i];
+    if (j >= pe) continue;
     if (PASS == 2) {
       if ((o >> 21) == pre) atomicAdd(&s_h[(o >> 10) & 2047u], 1u);
     } else {
@@ -443,6 +506,7 @@ __global__ void __launch_bounds__(256) k_sel_hist(DevParams P) {
 __global__ void __launch_bounds__(256) k_sel_count(DevParams P) {
   __shared__ unsigned s_warp[32];
   const int u = blockIdx.x, seg = blockIdx.y;
+  grid_dependency_wait();
   const UnitInfo inf = P.info[u];
   if (inf.k <= 0) return;
   const int pb = inf.s1 + seg * kSeg;
@@ -453,10 +517,20 @@ __global__ void __launch_bounds__(256) k_sel_count(DevParams P) {
                        static_cast<unsigned>(st.d3);
   const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
   unsigned gt = 0, eq = 0;
-  for (int j = pb + threadIdx.x; j < pe; j += blockDim.x) {
-    const unsigned o = ordk[j];
-    gt += o > thr;
-    eq += o == thr;
+  constexpr int PER = kSeg / 256;
+  unsigned keys[PER];
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    const int j = pb + threadIdx.x + 256 * i;
+    keys[i] = j < pe ? ordk[j] : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    const int j = pb + threadIdx.x + 256 * i;
+    if (j < pe) {
+      gt += keys[i] > thr;
+      eq += keys[i] == thr;
+    }
   }
   gt = block_sum(gt, s_warp);
   eq = block_sum(eq, s_warp);
@@ -477,6 +551,7 @@ __global__ void __launch_bounds__(256) k_sel_write(DevParams P) {
   __shared__ unsigned s_warp[32];
   __shared__ unsigned s_before[2];
   const int u = blockIdx.x, seg = blockIdx.y;
+  grid_dependency_wait();
   const UnitInfo inf = P.info[u];
   if (inf.k <= 0) return;
   const int pb = inf.s1 + seg * kSeg;
@@ -523,6 +598,183 @@ __global__ void __launch_bounds__(256) k_sel_write(DevParams P) {
     if (take[i]) sel[pos++] = j0 + i;
 }
 
+// ============================================================ k_select (cluster)
+// The whole top-k selection of one unit in one cluster of kSelCluster CTAs.
+// CTA r of the cluster owns a contiguous segment of the middle's keys, staged
+// once in its shared memory. Digits 2 and 3 of the radix select are found
+// from cluster-wide histograms: every CTA histograms its segment, CTA r sums
+// bin slice r over the cluster (distributed shared memory), and every CTA
+// gathers the summed slices. The counts above / equal to the threshold are
+// exchanged the same way, and each CTA compacts its segment in order. Phases
+// are separated by cluster barriers.
+constexpr int kSelCluster = 8;
+constexpr int kSelFixedSmem = (kHist2 + kHist2 / kSelCluster + kHist2) * 4 + 64;
+
+__device__ __forceinline__ unsigned* cluster_peer(unsigned* p, int rank) {
+  return cooperative_groups::this_cluster().map_shared_rank(p, rank);
+}
+
+// Cluster-wide histogram of NB bins from each CTA's s_loc; result in s_full.
+template <int NB>
+__device__ __forceinline__ void cluster_hist_allreduce(unsigned* s_loc, unsigned* s_red, unsigned* s_full,
+                                                       int rank) {
+  auto cluster = cooperative_groups::this_cluster();
+  constexpr int SL = NB / kSelCluster;  // bins summed by each CTA
+  cluster.sync();
+  for (int x = threadIdx.x; x < SL; x += blockDim.x) {
+    unsigned acc = 0;
+#pragma unroll
+    for (int q = 0; q < kSelCluster; q++) acc += cluster_peer(s_loc, q)[rank * SL + x];
+    s_red[x] = acc;
+  }
+  cluster.sync();
+  for (int x = threadIdx.x; x < NB; x += blockDim.x) s_full[x] = cluster_peer(s_red, x / SL)[x % SL];
+  cluster.sync();  // s_red and s_loc may be reused after every CTA gathered
+}
+
+__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(256) k_select(DevParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned* s_loc = reinterpret_cast<unsigned*>(smem);  // [kHist2] local histogram
+  unsigned* s_red = s_loc + kHist2;                      // [kHist2 / cluster] summed slice
+  unsigned* s_full = s_red + kHist2 / kSelCluster;       // [kHist2] cluster histogram
+  unsigned* s_cnt = s_full + kHist2;                     // [2] this CTA's counts above / equal
+  unsigned* s_keys = reinterpret_cast<unsigned*>(smem + kSelFixedSmem);
+  __shared__ unsigned s_warp[32];
+  __shared__ int s_digit, s_krem;
+  auto cluster = cooperative_groups::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int u = blockIdx.x / kSelCluster;
+  grid_dependency_wait();
+  const UnitInfo inf = P.info[u];
+  if (inf.k <= 0) return;  // uniform over the cluster: no peer touches this CTA
+  const int mlen = inf.wst - inf.s1;
+  const int seglen = (mlen + kSelCluster - 1) / kSelCluster;
+  const int pb = inf.s1 + rank * seglen;
+  const int pe = min(inf.wst, pb + seglen);
+  const int cnt = max(0, pe - pb);
+  const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
+  for (int base = 0; base < cnt; base += 16 * 256) {  // 16 independent loads in flight per thread
+    unsigned v[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const int x = base + i * 256 + threadIdx.x;
+      v[i] = x < cnt ? ordk[pb + x] : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const int x = base + i * 256 + threadIdx.x;
+      if (x < cnt) s_keys[x] = v[i];
+    }
+  }
+  __syncthreads();
+
+  // digit 1 from the score pass's histogram (every CTA resolves it)
+  if (threadIdx.x == 0) {
+    s_digit = 0;
+    s_krem = inf.k;
+  }
+  __syncthreads();
+  const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHistAll;
+  find_digit<kHist1>(h1, inf.k, &s_digit, &s_krem, s_warp);
+  const unsigned d1 = static_cast<unsigned>(s_digit);
+  const int krem1 = s_krem;
+
+  // digit 2
+  for (int x = threadIdx.x; x < kHist2; x += blockDim.x) s_loc[x] = 0u;
+  __syncthreads();
+  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
+    const unsigned o = s_keys[x];
+    if ((o >> 21) == d1) atomicAdd(&s_loc[(o >> 10) & 2047u], 1u);
+  }
+  cluster_hist_allreduce<kHist2>(s_loc, s_red, s_full, rank);
+  find_digit<kHist2>(s_full, krem1, &s_digit, &s_krem, s_warp);
+  const unsigned d2 = static_cast<unsigned>(s_digit);
+  const int krem2 = s_krem;
+
+  // digit 3
+  const unsigned pre = d1 << 11 | d2;
+  for (int x = threadIdx.x; x < kHist3; x += blockDim.x) s_loc[x] = 0u;
+  __syncthreads();
+  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
+    const unsigned o = s_keys[x];
+    if ((o >> 10) == pre) atomicAdd(&s_loc[o & 1023u], 1u);
+  }
+  cluster_hist_allreduce<kHist3>(s_loc, s_red, s_full, rank);
+  find_digit<kHist3>(s_full, krem2, &s_digit, &s_krem, s_warp);
+  const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
+  const unsigned need_eq = static_cast<unsigned>(s_krem);
+
+  // counts above / equal per CTA, exchanged over the cluster
+  unsigned gt = 0, eq = 0;
+  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
+    const unsigned o = s_keys[x];
+    gt += o > thr;
+    eq += o == thr;
+  }
+  gt = block_sum(gt, s_warp);
+  eq = block_sum(eq, s_warp);
+  if (threadIdx.x == 0) {
+    s_cnt[0] = gt;
+    s_cnt[1] = eq;
+  }
+  cluster.sync();
+  unsigned gt_before = 0, eq_before = 0;
+  for (int q = 0; q < rank; q++) {
+    const unsigned* pc = cluster_peer(s_cnt, q);
+    gt_before += pc[0];
+    eq_before += pc[1];
+  }
+  if (rank == 0 && threadIdx.x == 0) {
+    P.info[u].thr = thr;
+    P.info[u].need_eq = static_cast<int>(need_eq);
+  }
+
+  // ordered compaction of the segment, 16 consecutive keys per thread per round
+  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+  unsigned taken = gt_before + min(eq_before, need_eq);
+  unsigned eq_seen = eq_before;
+  constexpr int PER = 16;
+  for (int base = 0; base < cnt; base += PER * 256) {
+    const int x0 = base + threadIdx.x * PER;
+    unsigned neq = 0;
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+      const int x = x0 + i;
+      neq += (x < cnt) && s_keys[x] == thr;
+    }
+    const unsigned eq_incl = block_inclusive_scan(neq, s_warp);
+    unsigned eq_rank = eq_seen + eq_incl - neq;
+    unsigned tk = 0;
+    bool take[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+      const int x = x0 + i;
+      const bool valid = x < cnt;
+      const unsigned o = valid ? s_keys[x] : 0u;
+      const bool e = valid && o == thr;
+      take[i] = valid && (o > thr || (e && eq_rank < need_eq));
+      eq_rank += e;
+      tk += take[i];
+    }
+    const unsigned tk_incl = block_inclusive_scan(tk, s_warp);
+    unsigned pos = taken + tk_incl - tk;
+#pragma unroll
+    for (int i = 0; i < PER; i++)
+      if (take[i]) sel[pos++] = pb + x0 + i;
+    // totals of this round for the next one (last thread holds the inclusive sums)
+    __shared__ unsigned s_round[2];
+    if (threadIdx.x == blockDim.x - 1) {
+      s_round[0] = eq_incl;
+      s_round[1] = tk_incl;
+    }
+    __syncthreads();
+    eq_seen += s_round[0];
+    taken += s_round[1];
+    __syncthreads();
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
 // ============================================================ tail positions
 // Position of the rho-th tail element (0-based, ascending) of M minus top-k:
 // s1 + rho + c, with c the number of top-k entries t_i with t_i - s1 - i <= rho.
@@ -530,7 +782,7 @@ __device__ __forceinline__ int tail_position(const int* topk, int k, int s1, int
   int lo = 0, hi = k;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if (topk[mid] - s1 - mid <= rho) lo = mid + 1; else hi = mid;
+    if (topk[mid] - s1 - mid <= rho) lo = mid + 1; else hi = mid;  // topk: shared or global memory
   }
   return s1 + rho + lo;
 }
@@ -561,61 +813,137 @@ __device__ __forceinline__ int item_position(const DevParams& P, int u, const Un
   return tail_position(topk, inf.k, inf.s1, rho);
 }
 
-// ============================================================ k_pilot
-// True scores s = fl(dot(q_g, k_j) * scale) of every query head of the group,
-// for I_f and the p pilot draws, into pscore[u][i][g].
+// ============================================================ gathers
+// One kernel template, three modes, each a persistent grid over a flattened
+// list of items. Items are grouped in slices, two per unit (u, part): part 0
+// carries weight 1, part 1 is sample. pre[s] is the prefix of item counts
+// over slices s = 2u + part; CTA c of C owns items [c*T/C, (c+1)*T/C) of the
+// T in total and writes one record per slice it touches, at index c + s
+// (unique: along the flattened order both c and s only grow, and one of them
+// grows at every segment boundary).
+//   det:    part 0 = I_f (or all of I_f and the tail when the tail is no
+//           larger than the pilot); part 1 = the p pilot draws. True scores
+//           of every query head go to pscore; the unit's last CTA computes
+//           the budget; the grid's last CTA writes the sample prefix.
+//   sample: part 0 = the whole tail when the budget covers it; part 1 = the
+//           draws t in [p, b). The unit's last CTA merges its det and sample
+//           records and writes the output.
+//   dense:  part 0 = every position; the unit's last CTA writes the output.
+// Rows are staged by cp.async into a per-warp double buffer, so each warp
+// computes one chunk while the next chunk's rows are in flight.
+constexpr int kModeDet = 0, kModeSample = 1, kModeDense = 2;
+
+// Row-per-lane-pair gather: each pair of lanes of a warp owns one gathered row
+// of a batch of 16 (even lane: even 16-byte chunks, odd lane: odd chunks; the
+// halving tree over chunks pairs chunks of equal parity until its last add).
+// K and V rows are staged in shared memory, XOR-swizzled by chunk so lanes
+// reading the same logical chunk of different rows hit different banks. Each
+// lane also owns D/32 output dimensions of the value accumulation.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) k_pilot(DevParams P) {
-  constexpr int E = Elem<T>::kPer16;
-  constexpr int L = D / E;
-  constexpr int RPW = 32 / L;
-  __shared__ int s_topk[kTopkSmem];
-  const int u = blockIdx.x, a = blockIdx.y;
-  const UnitInfo inf = P.info[u];
-  if (inf.mode != 2) return;
-  const int nA = inf.nI + inf.p;
-  const int ib = static_cast<int>(static_cast<long long>(nA) * a / P.SA);
-  const int ie = static_cast<int>(static_cast<long long>(nA) * (a + 1) / P.SA);
-  if (ib >= ie) return;
-  const int* topk = stage_topk(P, u, inf, s_topk);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int grp = lane / L, li = lane % L;
-  const int b = u / P.Hkv, h = u % P.Hkv;
-  float q[G][E];
-#pragma unroll
-  for (int g = 0; g < G; g++)
-#pragma unroll
-    for (int e = 0; e < E; e++)
-      q[g][e] = Elem<T>::load(P.q, (static_cast<size_t>(b) * P.Hq + h * G + g) * D + li * E + e);
-  const T* kc = static_cast<const T*>(P.k);
-  float* ps = P.pscore + static_cast<size_t>(u) * P.max_ctx * G;
-  constexpr int UU = 2;
-  // warp-uniform trip count: every lane runs the shuffles of group_allreduce
-  for (int wb = ib + warp * RPW * UU; wb < ie; wb += nwarps * RPW * UU) {
-    uint4 raw[UU];
-#pragma unroll
-    for (int k = 0; k < UU; k++) {
-      const int i = wb + k * RPW + grp;
-      if (i < ie) {
-        const int j = item_position(P, u, inf, topk, i, false);
-        raw[k] = ld_gather(kc + row_off(P, b, h, j, D) + li * E);
-      } else {
-        raw[k] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < UU; k++) {
-      const int i = wb + k * RPW + grp;
-#pragma unroll
-      for (int g = 0; g < G; g++) {
-        const float s = __fmul_rn(group_allreduce<L>(chunk_dot<T>(q[g], raw[k])), P.scale);
-        if (li == 0 && i < ie) ps[static_cast<size_t>(i) * G + g] = s;
-      }
-    }
+struct GatherShape {
+  static constexpr int E = Elem<T>::kPer16;        // elements per 16-byte chunk
+  static constexpr int NC = D / E;                 // chunks per row
+  static constexpr int LOGNC = ilog2c(NC);
+  static constexpr int ROWB = D * static_cast<int>(sizeof(T));
+  static constexpr int DPL = D / 32;               // value dims per lane
+  static constexpr int NW = 8;                     // warps per CTA
+  static constexpr int BATCH = 16;                 // items per warp batch (one per lane pair)
+  static constexpr int STAGE = BATCH * 2 * ROWB;   // K rows then V rows of a batch
+  static constexpr int REC = G * (2 + D);          // floats per record: (m, l, acc[D]) per head
+  static constexpr size_t RED = static_cast<size_t>(NW) * G * D * 4;  // merge buffer (aliases the stages)
+  static constexpr size_t OFF_Q = (static_cast<size_t>(NW) * STAGE > RED ? static_cast<size_t>(NW) * STAGE : RED);
+  static constexpr size_t OFF_STAT = OFF_Q + static_cast<size_t>(G) * D * 4;  // [NW][G][2]
+  // dynamic shared memory; the sample gather appends its slice prefix
+  static constexpr size_t SMEM = OFF_STAT + static_cast<size_t>(NW) * G * 2 * 4;
+};
+
+// Byte offset of logical chunk c of row r in a swizzled batch area.
+template <int NC>
+__device__ __forceinline__ int swz(int r, int c) {
+  return (r * NC + (c ^ (r & (NC - 1)))) * 16;
+}
+
+__host__ __device__ constexpr int bitrev_c(int x, int bits) {
+  return bits == 0 ? 0 : ((x & 1) << (bits - 1)) | bitrev_c(x >> 1, bits - 1);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  const size_t g = __cvta_generic_to_global(gsrc);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(g) : "memory");
+}
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void l2_prefetch(const void* gsrc, int bytes) {
+  const size_t g = __cvta_generic_to_global(gsrc);  // the instruction takes a global-space address
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(g), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// CTA of C holding flattened item x of T (CTA c owns [c*T/C, (c+1)*T/C)).
+__device__ __forceinline__ int cta_of(long long x, long long T, int C) {
+  return static_cast<int>(((x + 1) * C - 1) / T);
+}
+
+// Item counts of unit u's two slices in a mode (from its validated state).
+template <int MODE>
+__device__ __forceinline__ void slice_counts(const UnitInfo& inf, int& n0, int& n1) {
+  if (MODE == kModeDense) {
+    n0 = inf.n;
+    n1 = 0;
+  } else if (MODE == kModeDet) {
+    const int n_extra = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
+    const int n_det = inf.mode == 2 ? inf.nI : inf.nI + n_extra;
+    n0 = n_det;
+    n1 = inf.nI + n_extra - n_det;
+  } else {
+    const bool whole_tail = inf.mode == 2 && inf.exhausted;
+    const bool sampled = inf.mode == 2 && !inf.exhausted;
+    n0 = whole_tail ? inf.ntail : 0;
+    n1 = sampled ? inf.bsz - inf.p : 0;
   }
 }
 
-// ============================================================ k_budget
+// Exclusive prefix over 2*units slice counts into pre[0 .. 2*units] (one CTA).
+template <int MODE>
+__device__ void write_slice_prefix(const DevParams& P, long long* pre, unsigned* s_warp,
+                                   long long* s_carry) {
+  if (threadIdx.x == 0) *s_carry = 0;
+  __syncthreads();
+  const int ns = 2 * P.units;
+  for (int base = 0; base < ns; base += blockDim.x) {
+    const int sidx = base + threadIdx.x;
+    unsigned cnt = 0;
+    if (sidx < ns) {
+      const UnitInfo inf = P.info[sidx >> 1];
+      int n0, n1;
+      slice_counts<MODE>(inf, n0, n1);
+      cnt = static_cast<unsigned>((sidx & 1) ? n1 : n0);
+    }
+    const long long carry = *s_carry;
+    const unsigned incl = block_inclusive_scan(cnt, s_warp);  // a 256-slice chunk sum fits in 32 bits
+    if (sidx < ns) pre[sidx] = carry + (incl - cnt);
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) *s_carry = carry + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) pre[ns] = *s_carry;
+}
+
+// Records of slice s: CTAs [c_first, c_last] (empty when c_first > c_last).
+__device__ __forceinline__ void slice_ctas(const long long* pre, int s, long long T, int C, int& cf,
+                                           int& cl) {
+  if (pre[s + 1] <= pre[s]) {
+    cf = 1;
+    cl = 0;
+    return;
+  }
+  cf = cta_of(pre[s], T, C);
+  cl = cta_of(pre[s + 1] - 1, T, C);
+}
+
+// ============================================================ budget
 struct U128 {
   unsigned long long lo, hi;
 };
@@ -625,7 +953,6 @@ __device__ __forceinline__ U128 u128_add(U128 a, U128 b) {
   r.hi = a.hi + b.hi + (r.lo < a.lo ? 1ull : 0ull);
   return r;
 }
-
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -642,23 +969,24 @@ __device__ __forceinline__ U128 warp_sum_u128(U128 v) {
   return v;
 }
 
-// Per query head: m = max score over I_f and the pilot; x = vexp(s - m);
-// xq = round(x * 2^32); S_f = sum over I_f, S1 and S2 = sums of xq and xq^2
-// over the pilot (integers, so the reduction order does not matter);
+// Per query head: m = max true score over I_f and the pilot (s_mh, from the
+// unit's det records: the same fp32 scores, so exact); x = vexp(s - m);
+// xq = round(x * 2^32); S_f = sum of xq over I_f, S1 and S2 = sums of xq and
+// xq^2 over the pilot (integers, so the reduction order does not matter);
 // n_h = (z * N_tail * sigma / (eps * D))^2 with sigma^2 = (p S2 - S1^2) /
-// (p (p - 1)) and D = S_f + N_tail * S1 / p, evaluated in double in a fixed
-// operation order. b = max(p, max_h n_h); b >= N_tail takes the whole tail.
+// (p (p - 1)) and D = S_f + N_tail * S1 / p, in double in a fixed operation
+// order. b = max(p, max_h n_h); b >= N_tail takes the whole tail instead.
+// Block of 256 threads.
 template <int G>
-__global__ void __launch_bounds__(256) k_budget(DevParams P) {
-  __shared__ float s_m[8];
-  __shared__ unsigned long long s_a[8], s_b[8];
-  __shared__ U128 s_c[8];
+__device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, const float* ps,
+                            const float* s_mh) {
+  __shared__ unsigned long long s_a[8][G], s_b[8][G];
+  __shared__ U128 s_c[8][G];
   __shared__ int s_need[G];
-  const int u = blockIdx.x;
   const int b = u / P.Hkv, h = u % P.Hkv;
-  UnitInfo inf = P.info[u];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   if (inf.mode != 2) {
+    __syncthreads();
     if (tid == 0) {
       const int bsz = inf.mode == 1 ? inf.ntail : 0;
       P.info[u].bsz = bsz;
@@ -668,70 +996,92 @@ __global__ void __launch_bounds__(256) k_budget(DevParams P) {
       P.sel_count[u] = inf.nI + bsz;
     }
     if (tid < G) P.head_need[static_cast<size_t>(b) * P.Hq + h * G + tid] = inf.mode == 1 ? inf.ntail : 0;
+    __syncthreads();
     return;
   }
-  const int nA = inf.nI + inf.p;
-  const float* ps = P.pscore + static_cast<size_t>(u) * P.max_ctx * G;
-  for (int g = 0; g < G; g++) {
-    float m = -INFINITY;
-    for (int i = tid; i < nA; i += blockDim.x) m = fmaxf(m, ps[static_cast<size_t>(i) * G + g]);
+  float mh[G];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_m[warp] = m;
-    __syncthreads();
-    m = s_m[0];
-    for (int w = 1; w < nw; w++) m = fmaxf(m, s_m[w]);
-    unsigned long long sf = 0, s1 = 0;
-    U128 s2{0ull, 0ull};
-    for (int i = tid; i < nA; i += blockDim.x) {
-      const float x = vexp(__fsub_rn(ps[static_cast<size_t>(i) * G + g], m));
-      const unsigned long long xq = __float2ull_rn(__fmul_rn(x, 4294967296.0f));
-      if (i < inf.nI) {
-        sf += xq;
-      } else {
-        s1 += xq;
-        s2 = u128_add(s2, U128{xq * xq, __umul64hi(xq, xq)});
-      }
-    }
-    sf = warp_sum_u64(sf);
-    s1 = warp_sum_u64(s1);
-    s2 = warp_sum_u128(s2);
-    __syncthreads();
-    if (lane == 0) {
-      s_a[warp] = sf;
-      s_b[warp] = s1;
-      s_c[warp] = s2;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      unsigned long long Sf = 0, S1 = 0;
-      U128 S2{0ull, 0ull};
-      for (int w = 0; w < nw; w++) {
-        Sf += s_a[w];
-        S1 += s_b[w];
-        S2 = u128_add(S2, s_c[w]);
-      }
-      const unsigned long long p = static_cast<unsigned long long>(inf.p);
-      // V = p*S2 - S1^2 (exact, >= 0)
-      U128 pS2;
-      pS2.lo = p * S2.lo;
-      pS2.hi = __umul64hi(p, S2.lo) + p * S2.hi;
-      const unsigned long long sq_lo = S1 * S1, sq_hi = __umul64hi(S1, S1);
-      U128 V;
-      V.lo = pS2.lo - sq_lo;
-      V.hi = pS2.hi - sq_hi - (pS2.lo < sq_lo ? 1ull : 0ull);
-      const double Vd = __dadd_rn(__dmul_rn(__ull2double_rn(V.hi), 18446744073709551616.0),
-                                  __ull2double_rn(V.lo));
-      const double pd = static_cast<double>(inf.p);
-      const double var = __ddiv_rn(Vd, __dmul_rn(pd, static_cast<double>(inf.p - 1)));
-      const double nt = static_cast<double>(inf.ntail);
-      const double Dq = __dadd_rn(__ull2double_rn(Sf), __ddiv_rn(__dmul_rn(nt, __ull2double_rn(S1)), pd));
-      const double t = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), Dq));
-      const double need = __dmul_rn(__dmul_rn(t, t), var);
-      s_need[g] = need >= nt ? inf.ntail : static_cast<int>(ceil(need));
-    }
-    __syncthreads();
+  for (int g = 0; g < G; g++) mh[g] = s_mh[g];
+  const int nA = inf.nI + inf.p;
+  unsigned long long sf[G], s1[G];
+  U128 s2[G];
+#pragma unroll
+  for (int g = 0; g < G; g++) {
+    sf[g] = s1[g] = 0ull;
+    s2[g] = U128{0ull, 0ull};
   }
+  constexpr int BATCH = 4;
+  for (int i0 = tid; i0 < nA; i0 += BATCH * 256) {
+    float sv[BATCH][G];
+#pragma unroll
+    for (int k = 0; k < BATCH; k++) {
+      const int i = i0 + k * 256;
+#pragma unroll
+      for (int g = 0; g < G; g++) sv[k][g] = i < nA ? ps[static_cast<size_t>(i) * G + g] : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; k++) {
+      const int i = i0 + k * 256;
+      if (i >= nA) continue;
+#pragma unroll
+      for (int g = 0; g < G; g++) {
+        const float x = vexp(__fsub_rn(sv[k][g], mh[g]));
+        const unsigned long long xq = __float2ull_rn(__fmul_rn(x, 4294967296.0f));
+        if (i < inf.nI) {
+          sf[g] += xq;
+        } else {
+          s1[g] += xq;
+          s2[g] = u128_add(s2[g], U128{xq * xq, __umul64hi(xq, xq)});
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; g++) {
+    sf[g] = warp_sum_u64(sf[g]);
+    s1[g] = warp_sum_u64(s1[g]);
+    s2[g] = warp_sum_u128(s2[g]);
+  }
+  __syncthreads();
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+      s_a[warp][g] = sf[g];
+      s_b[warp][g] = s1[g];
+      s_c[warp][g] = s2[g];
+    }
+  }
+  __syncthreads();
+  if (tid < G) {
+    const int g = tid;
+    unsigned long long Sf = 0, S1 = 0;
+    U128 S2{0ull, 0ull};
+    for (int w = 0; w < nw; w++) {
+      Sf += s_a[w][g];
+      S1 += s_b[w][g];
+      S2 = u128_add(S2, s_c[w][g]);
+    }
+    const unsigned long long p = static_cast<unsigned long long>(inf.p);
+    U128 pS2;  // p * S2, exact
+    pS2.lo = p * S2.lo;
+    pS2.hi = __umul64hi(p, S2.lo) + p * S2.hi;
+    const unsigned long long sq_lo = S1 * S1, sq_hi = __umul64hi(S1, S1);
+    U128 V;    // p * S2 - S1^2 >= 0
+    V.lo = pS2.lo - sq_lo;
+    V.hi = pS2.hi - sq_hi - (pS2.lo < sq_lo ? 1ull : 0ull);
+    const double Vd = __dadd_rn(__dmul_rn(__ull2double_rn(V.hi), 18446744073709551616.0),
+                                __ull2double_rn(V.lo));
+    const double pd = static_cast<double>(inf.p);
+    const double var = __ddiv_rn(Vd, __dmul_rn(pd, static_cast<double>(inf.p - 1)));
+    const double nt = static_cast<double>(inf.ntail);
+    const double Dq = __dadd_rn(__ull2double_rn(Sf), __ddiv_rn(__dmul_rn(nt, __ull2double_rn(S1)), pd));
+    const double t = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), Dq));
+    const double need = __dmul_rn(__dmul_rn(t, t), var);
+    const int nh = need >= nt ? inf.ntail : static_cast<int>(ceil(need));
+    s_need[g] = nh;
+    P.head_need[static_cast<size_t>(b) * P.Hq + h * G + g] = nh;
+  }
+  __syncthreads();
   if (tid == 0) {
     int nmax = 0;
     for (int g = 0; g < G; g++) nmax = max(nmax, s_need[g]);
@@ -747,213 +1097,485 @@ __global__ void __launch_bounds__(256) k_budget(DevParams P) {
     P.budgets[u] = bsz;
     P.sel_count[u] = inf.nI + bsz;
   }
-  if (tid < G) P.head_need[static_cast<size_t>(b) * P.Hq + h * G + tid] = s_need[tid];
+  __syncthreads();
+}
+
+// Max score per head over unit u's det records (both parts) into s_mh. The
+// record maxima are loaded by all threads at once, then reduced.
+template <int D, int G>
+__device__ void det_record_max(const DevParams& P, int u, float* s_mh, float* s_scr) {
+  constexpr int REC = G * (2 + D);
+  const long long T = P.pre_det[2 * P.units];
+  int cf0, cl0, cf1, cl1;
+  slice_ctas(P.pre_det, 2 * u, T, P.CD, cf0, cl0);
+  slice_ctas(P.pre_det, 2 * u + 1, T, P.CD, cf1, cl1);
+  const int n0 = max(0, cl0 - cf0 + 1), n1 = max(0, cl1 - cf1 + 1);
+  for (int x = threadIdx.x; x < (n0 + n1) * G; x += blockDim.x) {
+    const int r = x / G, g = x % G;
+    const size_t id = r < n0 ? static_cast<size_t>(cf0 + r + 2 * u) : static_cast<size_t>(cf1 + (r - n0) + 2 * u + 1);
+    s_scr[x] = P.rec_det[id * REC + g * (2 + D)];
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float m = -INFINITY;
+    for (int r = 0; r < n0 + n1; r++) m = fmaxf(m, s_scr[r * G + threadIdx.x]);
+    s_mh[threadIdx.x] = m;
+  }
+  __syncthreads();
+}
+
+// out = (A_0 + w A_1) / (L_0 + w L_1) for unit u from its records, with part 1
+// weighted by w = N_tail / b when the tail was sampled (1 otherwise). Block of
+// 256 threads; s_scr holds SCR floats (P.combine_scr when SCR is 0). A flat
+// table of the unit's records is built first; every record's (m, l) is then
+// loaded by all threads at once; maxima and scale factors come from shared
+// memory, and each output element sums its records' accumulators.
+template <int D, int G, int MODE, int SCR>
+__device__ void unit_combine(const DevParams& P, int u, float* s_scr) {
+  constexpr int REC = G * (2 + D);
+  __shared__ int s_tot;
+  const UnitInfo inf = P.info[u];
+  const int b = u / P.Hkv, h = u % P.Hkv;
+  const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
+  const bool sampled = MODE == kModeSample && inf.mode == 2 && !inf.exhausted;
+  const int scr = SCR > 0 ? SCR : P.combine_scr;
+  // scratch layout: record table [tot] (offset in floats, part in the low bit
+  // of a separate int array), then (m, l) [tot][G][2], scale factors [tot][G],
+  // and M, L [2][G] at the end
+  long long* s_roff = reinterpret_cast<long long*>(s_scr);
+  float* s_M = s_scr + scr - 4 * G;
+  float* s_L = s_M + 2 * G;
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    const long long Tm = (MODE == kModeSample) ? P.pre_samp[2 * P.units] : P.pre_det[2 * P.units];
+    const long long Td = P.pre_det[2 * P.units];
+    for (int part = 0; part < 2; part++) {
+      int cf, cl;
+      // this kernel's records (the sample gather's, or the dense/det gather's)
+      slice_ctas(MODE == kModeSample ? P.pre_samp : P.pre_det, 2 * u + part, Tm,
+                 MODE == kModeSample ? P.CS : P.CD, cf, cl);
+      const float* base = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
+      const long long bo = base == P.rec_det ? 0 : (P.rec_samp - P.rec_det);
+      for (int c = cf; c <= cl; c++) s_roff[tot++] = ((bo + static_cast<long long>(c + 2 * u + part) * REC) << 1) | part;
+      // the det gather's records, in sample mode (the pilot is dropped when the
+      // whole tail is taken)
+      if (MODE == kModeSample && !(part == 1 && whole_tail)) {
+        slice_ctas(P.pre_det, 2 * u + part, Td, P.CD, cf, cl);
+        for (int c = cf; c <= cl; c++) s_roff[tot++] = (static_cast<long long>(c + 2 * u + part) * REC) << 1 | part;
+      }
+    }
+    s_tot = tot;
+  }
+  __syncthreads();
+  const int tot = s_tot;
+  float* s_ml = s_scr + 2 * tot;          // after the table (tot long longs)
+  float* s_cf = s_ml + 2 * tot * G;
+  for (int x = threadIdx.x; x < tot * G * 2; x += blockDim.x) {
+    const int r = x / (2 * G), g = (x / 2) % G, f = x & 1;
+    s_ml[x] = P.rec_det[(s_roff[r] >> 1) + g * (2 + D) + f];
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * G) {
+    const int part = threadIdx.x / G, g = threadIdx.x % G;
+    float M = -INFINITY;
+    for (int r = 0; r < tot; r++)
+      if ((s_roff[r] & 1) == part) M = fmaxf(M, s_ml[(r * G + g) * 2]);
+    float Lsum = 0.0f;
+    for (int r = 0; r < tot; r++) {
+      if ((s_roff[r] & 1) != part) continue;
+      const float mr = s_ml[(r * G + g) * 2];
+      const float c = (mr == -INFINITY) ? 0.0f : __expf(mr - M);
+      s_cf[r * G + g] = c;
+      Lsum += s_ml[(r * G + g) * 2 + 1] * c;
+    }
+    s_M[part * G + g] = M;
+    s_L[part * G + g] = Lsum;
+  }
+  __syncthreads();
+  float w = 1.0f;
+  if (sampled) w = static_cast<float>(static_cast<double>(inf.ntail) / static_cast<double>(inf.bsz));
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, e = idx % D;
+    float* out = P.out + (static_cast<size_t>(b) * P.Hq + h * G + g) * D + e;
+    if (inf.n <= 0) {
+      *out = 0.0f;
+      continue;
+    }
+    float A0 = 0.0f, A1 = 0.0f;
+#pragma unroll 4
+    for (int r = 0; r < tot; r++) {
+      const long long ro = s_roff[r];
+      const float c = s_cf[r * G + g];
+      const float v = (c != 0.0f) ? P.rec_det[(ro >> 1) + g * (2 + D) + 2 + e] * c : 0.0f;
+      if (ro & 1) A1 += v; else A0 += v;
+    }
+    const float M0 = s_M[g], M1 = s_M[G + g];
+    const float M = fmaxf(M0, M1);
+    const float c0 = (M0 == -INFINITY) ? 0.0f : __expf(M0 - M);
+    const float c1 = (M1 == -INFINITY) ? 0.0f : __expf(M1 - M);
+    *out = (A0 * c0 + w * (A1 * c1)) / (s_L[g] * c0 + w * (s_L[G + g] * c1));
+  }
+  __syncthreads();
+}
+
+// Number of (CTA, slice) segments of unit u in this kernel.
+__device__ __forceinline__ int unit_segments(const long long* pre, int u, long long T, int C) {
+  int n = 0;
+  for (int part = 0; part < 2; part++) {
+    int cf, cl;
+    slice_ctas(pre, 2 * u + part, T, C, cf, cl);
+    n += max(0, cl - cf + 1);
+  }
+  return n;
 }
 
 // ============================================================ k_gather
-// Split-K softmax-and-accumulate over a contiguous slice [ib, ie) of unit u's
-// selected list (all positions, for dense). Entries below nDet carry weight 1
-// (I_f, or everything when the tail is taken whole); the rest are sample
-// draws. Each part keeps its own softmax state per query head: running max m,
-// exp sum l and exp-weighted value sum acc. The slice's two states go to
-// partial slot [u][blockIdx.y] as (m_f, l_f, m_s, l_s, acc_f[D], acc_s[D]).
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) k_gather(DevParams P) {
-  constexpr int E = Elem<T>::kPer16;
-  constexpr int L = D / E;
-  constexpr int RPW = 32 / L;
-  constexpr int NGRP = 8 * RPW;  // lane groups per CTA (8 warps)
-  constexpr int PW = 4 + 2 * D;  // floats per head in a partial
-  constexpr int UU = 2;          // rows in flight per lane group
-  __shared__ int s_topk[kTopkSmem];
-  __shared__ float s_stat[NGRP][G][2];
-  __shared__ float s_acc[G][D];
+template <typename T, int D, int G, int MODE>
+__global__ void __launch_bounds__(256, (G >= 8 ? 2 : 3)) k_gather(DevParams P) {
+  using S = GatherShape<T, D, G>;
+  constexpr int E = S::E, NC = S::NC, LOGNC = S::LOGNC, DPL = S::DPL, NW = S::NW;
+  constexpr int DB = DPL * static_cast<int>(sizeof(T));  // value bytes per lane (4, 8 or 16)
+  extern __shared__ __align__(128) unsigned char smem[];
+  float* s_q = reinterpret_cast<float*>(smem + S::OFF_Q);
+  float* s_red = reinterpret_cast<float*>(smem);  // aliases the stages during merges
+  float* s_stat = reinterpret_cast<float*>(smem + S::OFF_STAT);
+  __shared__ unsigned s_warp[32];
+  __shared__ long long s_carry;
 
-  const int u = blockIdx.x, a = blockIdx.y;
-  const UnitInfo inf = P.info[u];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int grp = lane / L, li = lane % L;
-  const int gid = warp * RPW + grp;
-  const int b = u / P.Hkv, h = u % P.Hkv;
-
-  const int n_items = P.dense ? inf.n : inf.nitems;
-  const bool whole_tail = inf.exhausted != 0;
-  const int n_det = (P.dense || whole_tail) ? n_items : inf.nI;
-  const int ib = static_cast<int>(static_cast<long long>(n_items) * a / P.SB);
-  const int ie = static_cast<int>(static_cast<long long>(n_items) * (a + 1) / P.SB);
-  const int* topk = s_topk;
-  if (!P.dense && ie > inf.nI && ib < ie) topk = stage_topk(P, u, inf, s_topk);
-
-  float q[G][E];
-#pragma unroll
-  for (int g = 0; g < G; g++)
-#pragma unroll
-    for (int e = 0; e < E; e++)
-      q[g][e] = Elem<T>::load(P.q, (static_cast<size_t>(b) * P.Hq + h * G + g) * D + li * E + e);
-
+  const int row = lane >> 1, par = lane & 1;  // my row in the batch, my chunk parity
+  grid_dependency_wait();
+  long long* pre = (MODE == kModeSample) ? P.pre_samp : P.pre_det;
+  float* rec = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
+  const int C = gridDim.x, c = blockIdx.x;
+  if (MODE == kModeSample) {
+    // the sample slices follow from the budgets; every CTA derives the prefix
+    // (CTA 0's copy is the one later kernels read)
+    long long* dst = (c == 0) ? pre : reinterpret_cast<long long*>(smem + S::SMEM);
+    write_slice_prefix<kModeSample>(P, dst, s_warp, &s_carry);
+    __syncthreads();
+    pre = dst;
+  }
+  const long long Tt = pre[2 * P.units];
+  const long long beg = Tt * c / C, end = Tt * (c + 1) / C;
+  long long cur = beg;
+  int sidx = 0;
+  if (beg < end) {
+    int lo = 0, hi = 2 * P.units;  // largest s with pre[s] <= beg
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= beg) lo = mid; else hi = mid;
+    }
+    sidx = lo;
+  }
   const T* kc = static_cast<const T*>(P.k);
   const T* vc = static_cast<const T*>(P.v);
-  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
-  float* part = P.partial + (static_cast<size_t>(u) * kSbMax + a) * G * PW;
+  unsigned char* kb_s = smem + warp * S::STAGE;          // this warp's K rows
+  unsigned char* vb_s = kb_s + S::BATCH * S::ROWB;       // and V rows
 
-#pragma unroll 1
-  for (int half = 0; half < 2; half++) {
-    const int rb = half == 0 ? ib : max(ib, n_det);
-    const int re = half == 0 ? min(ie, n_det) : ie;
-    float m[G], l[G], acc[G][E];
+  while (cur < end) {
+    while (pre[sidx + 1] <= cur) sidx++;
+    const long long send = min(end, pre[sidx + 1]);
+    const int u = sidx >> 1, part = sidx & 1;
+    const int lb = static_cast<int>(cur - pre[sidx]), le = static_cast<int>(send - pre[sidx]);
+    const UnitInfo inf = P.info[u];
+    const int b = u / P.Hkv, h = u % P.Hkv;
+    const bool valid = inf.n > 0;
+    const int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
+    const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
+    int n_det = 0;
+    if (MODE == kModeDet) {
+      int n0, n1;
+      slice_counts<kModeDet>(inf, n0, n1);
+      n_det = n0;
+    }
+    float* ps = (MODE == kModeDet && inf.mode == 2) ? P.pscore + static_cast<size_t>(u) * P.max_ctx * G
+                                                     : nullptr;
+    // local item l of this slice -> (item index i in the unit's list, cache
+    // position); positions of sampled entries were written by k_draws / k_budget
+    auto position = [&](int l, int& i) -> int {
+      if (MODE == kModeDense) {
+        i = l;
+        return l;
+      }
+      if (MODE == kModeDet) i = part == 0 ? l : n_det + l;
+      else i = inf.nI + (whole_tail ? l : inf.p + l);
+      return sel[i];
+    };
+
+    // queries of the group, fp32, in shared memory
+    __syncthreads();
+    for (int x = threadIdx.x; x < G * D; x += blockDim.x)
+      s_q[x] = Elem<T>::load(P.q, (static_cast<size_t>(b) * P.Hq + h * G) * D + x);
+    __syncthreads();
+
+    float m[G], l[G], acc[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; g++) {
       m[g] = -INFINITY;
       l[g] = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; e++) acc[g][e] = 0.0f;
+      for (int d = 0; d < DPL; d++) acc[g][d] = 0.0f;
     }
-    // warp-uniform trip count: every lane runs the shuffles of group_allreduce
-    for (int wb = rb + warp * RPW * UU; wb < re; wb += NGRP * UU) {
-      uint4 kr[UU], vr[UU];
-      bool ok[UU];
+    const int nitems = valid ? le - lb : 0;
+    const int nbatch = (nitems + S::BATCH - 1) / S::BATCH;
+    auto prefetch_rows = [&](int kbn) {  // next batch's rows into L2
+      const int xn = kbn + row;
+      if (kbn < nitems && xn < nitems && par == 0) {
+        int i2;
+        const size_t o2 = row_off(P, b, h, position(lb + xn, i2), D);
+        l2_prefetch(kc + o2, S::ROWB);
+        l2_prefetch(vc + o2, S::ROWB);
+      }
+    };
+
+    for (int kbi = warp; kbi < nbatch; kbi += NW) {
+      const int kb = kbi * S::BATCH;
+      const int x = kb + row;
+      const bool ok = x < nitems;
+      int item = 0;
+      long long off = 0;
+      if (ok && par == 0) {
+        const int pos = position(lb + x, item);
+        off = static_cast<long long>(row_off(P, b, h, pos, D));
+      }
+      off = __shfl_sync(0xffffffffu, off, lane & ~1);
+      prefetch_rows(kb + NW * S::BATCH);
+      if (ok) {
 #pragma unroll
-      for (int k = 0; k < UU; k++) {
-        const int i = wb + k * RPW + grp;
-        ok[k] = i < re;
-        if (ok[k]) {
-          int j = i;
-          if (!P.dense) {
-            j = item_position(P, u, inf, topk, i, whole_tail);
-            if (i >= inf.nI && li == 0) sel[i] = j;
+        for (int jj = 0; jj < NC / 2; jj++) {
+          const int cc = 2 * jj + par;
+          cp_async16(kb_s + swz<NC>(row, cc), kc + static_cast<size_t>(off) + cc * E);
+          cp_async16(vb_s + swz<NC>(row, cc), vc + static_cast<size_t>(off) + cc * E);
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncwarp();
+
+      // true scores of my row: my parity's chunk sums in bit-reversed order,
+      // merged as a binary counter (exactly the halving tree's pairs), then
+      // the tree's last add with the partner lane's half
+      float sc[G];
+      {
+        float st[G][LOGNC];
+#pragma unroll
+        for (int ii = 0; ii < NC / 2; ii++) {
+          const int cc = 2 * bitrev_c(ii, LOGNC - 1) + par;
+          const uint4 kr = *reinterpret_cast<const uint4*>(kb_s + swz<NC>(row, cc));
+          float kx[E];
+          Elem<T>::unpack(kr, kx);
+#pragma unroll
+          for (int g = 0; g < G; g++) {
+            const float* qg = s_q + g * D + cc * E;
+            float a = 0.0f;
+#pragma unroll
+            for (int e = 0; e < E; e++) a = __fmaf_rn(qg[e], kx[e], a);
+            int lev = 0;
+#pragma unroll
+            for (int bit = 0; bit < LOGNC - 1; bit++) {
+              if (((ii >> bit) & 1) == 0) break;
+              a = __fadd_rn(st[g][lev], a);
+              lev++;
+            }
+            st[g][lev] = a;
           }
-          const size_t off = row_off(P, b, h, j, D) + li * E;
-          kr[k] = ld_gather(kc + off);
-          vr[k] = ld_gather(vc + off);
-        } else {
-          kr[k] = vr[k] = make_uint4(0u, 0u, 0u, 0u);
         }
-      }
-      float s[UU][G];
-#pragma unroll
-      for (int k = 0; k < UU; k++)
-#pragma unroll
-        for (int g = 0; g < G; g++)
-          s[k][g] = __fmul_rn(group_allreduce<L>(chunk_dot<T>(q[g], kr[k])), P.scale);
-#pragma unroll
-      for (int g = 0; g < G; g++) {
-        float mx = m[g];
-#pragma unroll
-        for (int k = 0; k < UU; k++)
-          if (ok[k]) mx = fmaxf(mx, s[k][g]);
-        if (mx > m[g]) {
-          const float c = __expf(m[g] - mx);  // 0 while m = -inf
-          l[g] *= c;
-#pragma unroll
-          for (int e = 0; e < E; e++) acc[g][e] *= c;
-          m[g] = mx;
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < UU; k++) {
-        if (!ok[k]) continue;
-        float x[E];
-        Elem<T>::unpack(vr[k], x);
 #pragma unroll
         for (int g = 0; g < G; g++) {
-          const float e = __expf(s[k][g] - m[g]);
-          l[g] += e;
-#pragma unroll
-          for (int t = 0; t < E; t++) acc[g][t] = fmaf(e, x[t], acc[g][t]);
+          const float mine = st[g][LOGNC - 1];
+          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          sc[g] = ok ? __fmul_rn(__fadd_rn(mine, other), P.scale) : -INFINITY;
         }
       }
-    }
-
-    // ---- merge the CTA's lane groups into one state for this part
-    __syncthreads();
-    if (li == 0) {
+      if (ps != nullptr && ok && par == 0) {
+#pragma unroll
+        for (int g = 0; g < G; g++) ps[static_cast<size_t>(item) * G + g] = sc[g];
+      }
+      // online softmax over the batch (each row counted once, by its even lane)
+      float ew[G];
 #pragma unroll
       for (int g = 0; g < G; g++) {
-        s_stat[gid][g][0] = m[g];
-        s_stat[gid][g][1] = l[g];
-      }
-    }
-    __syncthreads();
+        float bm = sc[g];
 #pragma unroll
-    for (int g = 0; g < G; g++) {
-      float mm = -INFINITY;
-      for (int x = 0; x < NGRP; x++) mm = fmaxf(mm, s_stat[x][g][0]);
-      const float c = (m[g] == -INFINITY) ? 0.0f : __expf(m[g] - mm);
+        for (int o = 16; o >= 1; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        if (bm > m[g]) {
+          const float cc = __expf(m[g] - bm);  // 0 while m = -inf
+          l[g] *= cc;
 #pragma unroll
-      for (int e = 0; e < E; e++) {
-        float v = acc[g][e] * c;
-#pragma unroll
-        for (int o = L; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        acc[g][e] = v;
-      }
-      if (threadIdx.x == 0) {
-        float Lsum = 0.0f;
-        for (int x = 0; x < NGRP; x++) {
-          const float mx = s_stat[x][g][0];
-          Lsum += (mx == -INFINITY) ? 0.0f : s_stat[x][g][1] * __expf(mx - mm);
+          for (int d = 0; d < DPL; d++) acc[g][d] *= cc;
+          m[g] = bm;
         }
-        part[g * PW + 2 * half] = mm;
-        part[g * PW + 2 * half + 1] = Lsum;
+        ew[g] = ok ? __expf(sc[g] - m[g]) : 0.0f;
+        float es = par == 0 ? ew[g] : 0.0f;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) es += __shfl_xor_sync(0xffffffffu, es, o);
+        l[g] += es;
       }
-    }
-    // warps add their sums into s_acc one after another (fixed order)
-    for (int w = 0; w < 8; w++) {
-      if (warp == w && grp == 0) {
+      // value accumulation: lane owns dims [lane * DPL, (lane + 1) * DPL)
+      const int cnt = min(S::BATCH, nitems - kb);
+      const int vchunk = (lane * DB) >> 4, vin = (lane * DB) & 15;
+      for (int t = 0; t < cnt; t++) {
+        float et[G];
+#pragma unroll
+        for (int g = 0; g < G; g++) et[g] = __shfl_sync(0xffffffffu, ew[g], 2 * t);
+        const unsigned char* vp = vb_s + swz<NC>(t, vchunk) + vin;
+        float vx[DPL];
+        if (DB == 16) {
+          const uint4 w = *reinterpret_cast<const uint4*>(vp);
+          float tmp[E];
+          Elem<T>::unpack(w, tmp);
+#pragma unroll
+          for (int d = 0; d < DPL; d++) vx[d] = tmp[d];
+        } else if (DB == 8) {
+          const uint2 w = *reinterpret_cast<const uint2*>(vp);
+          if (sizeof(T) == 2) {
+            vx[0] = __uint_as_float(w.x << 16);
+            vx[1] = __uint_as_float(w.x & 0xFFFF0000u);
+            if (DPL > 2) {
+              vx[DPL > 2 ? 2 : 0] = __uint_as_float(w.y << 16);
+              vx[DPL > 3 ? 3 : 0] = __uint_as_float(w.y & 0xFFFF0000u);
+            }
+          } else {
+            vx[0] = __uint_as_float(w.x);
+            vx[DPL > 1 ? 1 : 0] = __uint_as_float(w.y);
+          }
+        } else {
+          const unsigned w = *reinterpret_cast<const unsigned*>(vp);
+          vx[0] = __uint_as_float(w << 16);
+          vx[DPL > 1 ? 1 : 0] = __uint_as_float(w & 0xFFFF0000u);
+        }
 #pragma unroll
         for (int g = 0; g < G; g++)
 #pragma unroll
-          for (int e = 0; e < E; e++) {
-            float& dst = s_acc[g][li * E + e];
-            dst = (w == 0) ? acc[g][e] : dst + acc[g][e];
-          }
+          for (int d = 0; d < DPL; d++) acc[g][d] = fmaf(et[g], vx[d], acc[g][d]);
       }
-      __syncthreads();
+      __syncwarp();
     }
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x)
-      part[(idx / D) * PW + 4 + half * D + idx % D] = s_acc[idx / D][idx % D];
+
+    // ---- merge the CTA's warps into one record for (CTA, slice)
+    __syncthreads();  // every warp is done with its stage (aliased by s_red)
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < G; g++) {
+        s_stat[(warp * G + g) * 2] = m[g];
+        s_stat[(warp * G + g) * 2 + 1] = l[g];
+      }
+    }
+    __syncthreads();
+    float* r = rec + static_cast<size_t>(c + sidx) * S::REC;
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+      float mb = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; w++) mb = fmaxf(mb, s_stat[(w * G + g) * 2]);
+      const float cw = (m[g] == -INFINITY) ? 0.0f : __expf(m[g] - mb);
+#pragma unroll
+      for (int d = 0; d < DPL; d++) s_red[(warp * G + g) * D + lane * DPL + d] = acc[g][d] * cw;
+      if (threadIdx.x == 0) {
+        float lb2 = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NW; w++) {
+          const float mw = s_stat[(w * G + g) * 2];
+          lb2 += (mw == -INFINITY) ? 0.0f : s_stat[(w * G + g) * 2 + 1] * __expf(mw - mb);
+        }
+        r[g * (2 + D)] = mb;
+        r[g * (2 + D) + 1] = lb2;
+      }
+    }
+    __syncthreads();
+    for (int x2 = threadIdx.x; x2 < G * D; x2 += blockDim.x) {
+      float a = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; w++) a += s_red[w * G * D + x2];
+      r[(x2 / D) * (2 + D) + 2 + x2 % D] = a;
+    }
+    cur = send;
   }
+  grid_dependents_launch();
+}
+
+// ============================================================ draw positions
+// Cache positions of unit u's sampled entries t in [t0, t1): with a sampled
+// tail, draw t is the Lemire map of Philox word t onto the tail; when the tail
+// is taken whole, entry t is the t-th tail position. Written to
+// sel[nI + t]. The sorted top-k list is staged in s_topk when it fits.
+__device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& inf, bool whole_tail,
+                                     int t0, int t1, int* s_topk) {
+  const int* g = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+  const int* topk = g;
+  if (inf.k <= kTopkSmem) {
+    for (int x = threadIdx.x; x < inf.k; x += blockDim.x) s_topk[x] = g[x];
+    __syncthreads();
+    topk = s_topk;
+  }
+  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
+  const unsigned bb = static_cast<unsigned>(u / P.Hkv), hh = static_cast<unsigned>(u % P.Hkv);
+  for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+    const int rho = whole_tail ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
+    sel[t] = tail_position(topk, inf.k, inf.s1, rho);
+  }
+  __syncthreads();
+}
+
+// ============================================================ k_draws
+// Positions of sampled entries, one thread per entry. PHASE 0 (before the det
+// gather): the p pilot draws, or the whole tail when it is no larger than the
+// pilot. PHASE 1 (after the budget): draws t in [p, b), or the whole tail
+// when the budget covers it. Grid (units, splits).
+template <int PHASE>
+__global__ void __launch_bounds__(256) k_draws(DevParams P) {
+  __shared__ int s_topk[kTopkSmem];
+  grid_dependency_wait();
+  const int u = blockIdx.x;
+  const UnitInfo inf = P.info[u];
+  int t0 = 0, t1 = 0;
+  bool whole = false;
+  if (PHASE == 0) {
+    if (inf.mode == 2) t1 = inf.p;
+    if (inf.mode == 1) {
+      t1 = inf.ntail;
+      whole = true;
+    }
+  } else if (inf.mode == 2) {
+    if (inf.exhausted) {
+      t1 = inf.ntail;
+      whole = true;
+    } else {
+      t0 = inf.p;
+      t1 = inf.bsz;
+    }
+  }
+  const int n = t1 - t0;
+  const int a = t0 + static_cast<int>(static_cast<long long>(n) * blockIdx.y / gridDim.y);
+  const int e = t0 + static_cast<int>(static_cast<long long>(n) * (blockIdx.y + 1) / gridDim.y);
+  if (a < e) write_draw_positions(P, u, inf, whole, a, e, s_topk);
+  grid_dependents_launch();
+}
+
+// ============================================================ k_budget
+// One CTA per unit: the per-head CLT budget from the det gather's records
+// (score maxima) and true scores.
+template <int D, int G>
+__global__ void __launch_bounds__(256) k_budget(DevParams P) {
+  __shared__ float s_mh[G];
+  extern __shared__ __align__(128) unsigned char smem[];
+  grid_dependency_wait();
+  const int u = blockIdx.x;
+  const UnitInfo inf = P.info[u];
+  if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh, reinterpret_cast<float*>(smem));
+  unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
+  grid_dependents_launch();
 }
 
 // ============================================================ k_combine
-// Per query head: merge the splits of each part to a common max, then
-// out = (A_f + w A_s) / (L_f + w L_s) with w = N_tail / b for a sampled tail
-// and 1 otherwise.
-template <int D, int G>
-__global__ void __launch_bounds__(1024) k_combine(DevParams P) {
-  constexpr int PW = 4 + 2 * D;
-  const int u = blockIdx.x;
-  const int b = u / P.Hkv, h = u % P.Hkv;
-  const int g = threadIdx.x / D, e = threadIdx.x % D;
-  if (g >= G) return;
-  const UnitInfo inf = P.info[u];
-  float* out = P.out + (static_cast<size_t>(b) * P.Hq + h * G + g) * D + e;
-  if (inf.n <= 0) {
-    *out = 0.0f;
-    return;
-  }
-  const float* part = P.partial + static_cast<size_t>(u) * kSbMax * G * PW + g * PW;
-  float Mh[2] = {-INFINITY, -INFINITY};
-  for (int a = 0; a < P.SB; a++)
-    for (int f = 0; f < 2; f++) Mh[f] = fmaxf(Mh[f], part[static_cast<size_t>(a) * G * PW + 2 * f]);
-  float Lh[2] = {0.f, 0.f}, Ah[2] = {0.f, 0.f};
-  for (int a = 0; a < P.SB; a++) {
-    const float* pa = part + static_cast<size_t>(a) * G * PW;
-    for (int f = 0; f < 2; f++) {
-      const float mx = pa[2 * f];
-      const float c = (mx == -INFINITY) ? 0.0f : __expf(mx - Mh[f]);
-      Lh[f] += pa[2 * f + 1] * c;
-      Ah[f] += pa[4 + f * D + e] * c;
-    }
-  }
-  const float M = fmaxf(Mh[0], Mh[1]);
-  const float cf = (Mh[0] == -INFINITY) ? 0.0f : __expf(Mh[0] - M);
-  const float cs = (Mh[1] == -INFINITY) ? 0.0f : __expf(Mh[1] - M);
-  float w = 1.0f;
-  if (!P.dense && inf.mode == 2 && !inf.exhausted)
-    w = static_cast<float>(static_cast<double>(inf.ntail) / static_cast<double>(inf.bsz));
-  const float num = Ah[0] * cf + w * (Ah[1] * cs);
-  const float den = Lh[0] * cf + w * (Lh[1] * cs);
-  *out = num / den;
+// One CTA per unit: merge its records and write the output.
+template <int D, int G, int MODE>
+__global__ void __launch_bounds__(256) k_combine(DevParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  grid_dependency_wait();
+  unit_combine<D, G, MODE, 0>(P, blockIdx.x, reinterpret_cast<float*>(smem));
+  grid_dependents_launch();
 }
 
 }  // namespace vattn
