@@ -70,7 +70,9 @@ enum {
   VATTN_OK = 0,
   VATTN_EINVAL = -1, /* a host argument is out of range or a required pointer is NULL */
   VATTN_ENOMEM = -2, /* workspace allocation failed in vattn_create                 */
-  VATTN_ECUDA = -3   /* a CUDA call or kernel launch failed                          */
+  VATTN_ECUDA = -3,  /* a CUDA call or kernel launch failed                          */
+  VATTN_ESCRATCH = -4 /* vattn_dense_decode_static: the call needs more scratch than
+                         its fixed device array holds                              */
 };
 
 /* bits of the device error word */
@@ -126,6 +128,31 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
 int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* page_table, const int32_t* seq_lens, int batch,
                        int num_pages, float* out, void* stream);
+
+/* Dense decode attention, as vattn_dense_decode, without a context and
+   without allocating anything. The paper has no counterpart: this entry point
+   serves callers that cannot allocate device memory when they call, e.g. a
+   server that has given all free memory to its KV-cache pool (an allocation
+   would fail), code that must not risk the device-wide wait that freeing
+   memory can cause, or a plug-in that cannot keep a context between calls.
+   `cfg` gives the shapes (proxy and proxy_rank are ignored); the other
+   arguments are those of vattn_dense_decode, on the current device.
+
+   Scratch: a fixed array of 8 MiB per device, defined in the library. A call
+   needs batch * Hq * (head_dim + 2) * 4 bytes of it at least; a larger call
+   returns VATTN_ESCRATCH before touching the device. The first call made with
+   a device current looks up that device's copy of the array (and its SM
+   count); make that first call before any stream capture begins. Every later
+   call on the device shares the same array: it keeps the last call's partial
+   results, nothing in it needs to start at zero (a call writes every part it
+   reads), and calls that overlap in time on one device race and corrupt
+   each other's output, so order them (one stream, or events). Device-side
+   violations (a page id out of range, a bad sequence length) give a zero
+   output for that sequence; there is no error word to read. */
+int vattn_dense_decode_static(const vattn_config* cfg, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* page_table,
+                              const int32_t* seq_lens, int batch, int num_pages, float* out,
+                              void* stream);
 
 /* sync != 0: wait for the device, then return and clear the device error
    word (VATTN_DEV_* bits). sync == 0: return the host status of the last

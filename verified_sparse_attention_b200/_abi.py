@@ -13,11 +13,12 @@ LIB_PATH = os.path.join(_HERE, "libvattn.so")
 
 VATTN_FP32, VATTN_BF16 = 0, 1
 VATTN_EXACT, VATTN_SPARQ, VATTN_LOKI = 0, 1, 2
-VATTN_OK, VATTN_EINVAL, VATTN_ENOMEM, VATTN_ECUDA = 0, -1, -2, -3
+VATTN_OK, VATTN_EINVAL, VATTN_ENOMEM, VATTN_ECUDA, VATTN_ESCRATCH = 0, -1, -2, -3, -4
 VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE = 1, 2
 
 # every symbol include/vattn.h declares
-EXPORTS = ("vattn_create", "vattn_decode", "vattn_dense_decode", "vattn_last_error",
+EXPORTS = ("vattn_create", "vattn_decode", "vattn_dense_decode", "vattn_dense_decode_static",
+           "vattn_last_error",
            "vattn_workspace_bytes", "vattn_set_timing", "vattn_score_pass_ms",
            "vattn_last_launch_count", "vattn_strerror", "vattn_destroy")
 
@@ -59,6 +60,8 @@ def lib():
         L.vattn_decode.restype = I
         L.vattn_dense_decode.argtypes = [P, P, P, P, P, P, I, I, P, P]
         L.vattn_dense_decode.restype = I
+        L.vattn_dense_decode_static.argtypes = [C.POINTER(vattn_config), P, P, P, P, P, I, I, P, P]
+        L.vattn_dense_decode_static.restype = I
         L.vattn_last_error.argtypes = [P, I]
         L.vattn_last_error.restype = I
         L.vattn_workspace_bytes.argtypes = [P]
@@ -124,6 +127,18 @@ def vattn_dense_decode(ctx, q, k_cache, v_cache, page_table, seq_lens, batch, nu
                                   _ptr(seq_lens), int(batch), int(num_pages), _ptr(out),
                                   _stream_ptr(stream))
     return _check(rc, "vattn_dense_decode") if check else rc
+
+
+def vattn_dense_decode_static(config, q, k_cache, v_cache, page_table, seq_lens, batch, num_pages,
+                              out, stream=None, check=True):
+    """Dense decode without a context or any allocation (scratch: a fixed
+    device array in the library, shared by every call on a device)."""
+    if isinstance(config, dict):
+        config = vattn_config(**config)
+    rc = lib().vattn_dense_decode_static(C.byref(config), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(page_table), _ptr(seq_lens), int(batch),
+                                         int(num_pages), _ptr(out), _stream_ptr(stream))
+    return _check(rc, "vattn_dense_decode_static") if check else rc
 
 
 def vattn_last_error(ctx, sync=True):

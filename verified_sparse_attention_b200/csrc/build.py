@@ -9,8 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(HERE, "vattn_api.cu")
-DEPS = [SRC, os.path.join(HERE, "vattn_kernels.cuh"), os.path.join(HERE, "vattn_device.cuh"),
+SRCS = [os.path.join(HERE, "vattn_api.cu"), os.path.join(HERE, "vattn_static.cu")]
+DEPS = [*SRCS, os.path.join(HERE, "vattn_kernels.cuh"), os.path.join(HERE, "vattn_device.cuh"),
         os.path.join(ROOT, "include", "vattn.h")]
 OUT = os.path.join(PKG, "libvattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -26,7 +26,7 @@ def needs_build():
 
 
 def build(verbose_ptxas=False, out=OUT):
-    cmd = [NVCC, *FLAGS, SRC, "-o", out]
+    cmd = [NVCC, *FLAGS, *SRCS, "-o", out]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.run(cmd, check=True)

@@ -227,6 +227,7 @@ const char* vattn_strerror(int code) {
     case VATTN_EINVAL: return "invalid argument";
     case VATTN_ENOMEM: return "device workspace allocation failed";
     case VATTN_ECUDA: return "CUDA call or kernel launch failed";
+    case VATTN_ESCRATCH: return "call needs more than the fixed 8 MiB scratch array of vattn_dense_decode_static";
     default: return "unknown code";
   }
 }
