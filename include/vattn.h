@@ -75,8 +75,9 @@ enum {
                          its fixed device array holds                              */
 };
 
-/* bits of the device error word */
-enum { VATTN_DEV_BAD_SEQLEN = 1, VATTN_DEV_BAD_PAGE = 2 };
+/* bits of the device error word; VATTN_DEV_TIMEOUT: a kernel's bounded wait
+   for its own copies ran out, so the call's outputs are not valid */
+enum { VATTN_DEV_BAD_SEQLEN = 1, VATTN_DEV_BAD_PAGE = 2, VATTN_DEV_TIMEOUT = 4 };
 
 typedef struct vattn_ctx vattn_ctx;
 

@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libvattn.so")
 VATTN_FP32, VATTN_BF16 = 0, 1
 VATTN_EXACT, VATTN_SPARQ, VATTN_LOKI = 0, 1, 2
 VATTN_OK, VATTN_EINVAL, VATTN_ENOMEM, VATTN_ECUDA, VATTN_ESCRATCH = 0, -1, -2, -3, -4
-VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE = 1, 2
+VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE, VATTN_DEV_TIMEOUT = 1, 2, 4
 
 # every symbol include/vattn.h declares
 EXPORTS = ("vattn_create", "vattn_decode", "vattn_dense_decode", "vattn_dense_decode_static",

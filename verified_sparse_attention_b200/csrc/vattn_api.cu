@@ -23,8 +23,8 @@ struct vattn_ctx {
   int nseg = 0;
   int score_grid = 0;
   int CD = 0, CS = 0;      // gather grid sizes (det/dense, sample)
-  size_t gather_smem = 0;   // det/dense gather
-  size_t sample_smem = 0;   // sample gather (adds its slice prefix)
+  size_t gather_smem = 0;   // gathers (all modes)
+  int gather_threads = 0;
   size_t budget_smem = 0;
   size_t combine_smem = 0;
   int combine_scr = 0;      // floats
@@ -93,6 +93,7 @@ struct Kernels {
   void (*combine_sample)(DevParams);
   void (*combine_dense)(DevParams);
   size_t gather_smem;
+  int gather_threads;
 };
 
 template <typename T, int D, int G>
@@ -109,6 +110,7 @@ Kernels kernels_for() {
   k.combine_sample = vattn::k_combine<D, G, vattn::kModeSample>;
   k.combine_dense = vattn::k_combine<D, G, vattn::kModeDense>;
   k.gather_smem = vattn::GatherShape<T, D, G>::SMEM;
+  k.gather_threads = vattn::GatherShape<T, D, G>::NW * 32;
   return k;
 }
 
@@ -261,12 +263,11 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
   ctx->score_grid = (occ < 1 ? 1 : occ) * ctx->num_sms;
   ctx->gather_smem = K.gather_smem;
-  ctx->sample_smem = K.gather_smem + (2 * U + 1) * sizeof(long long);
-  for (auto fn : {K.det, K.dense})
+  ctx->gather_threads = K.gather_threads;
+  for (auto fn : {K.det, K.sample, K.dense})
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->gather_smem));
-  cudaFuncSetAttribute(K.sample, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->sample_smem));
   int gocc = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, 256, ctx->sample_smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, K.gather_threads, ctx->gather_smem);
   if (gocc < 1) gocc = 1;
   ctx->CD = ctx->CS = gocc * ctx->num_sms;
   // the combine stages (m, l) and a scale factor per (record, head), and a
@@ -482,10 +483,10 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
   }
   launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
-  launch(K.det, dim3(ctx->CD), dim3(256), ctx->gather_smem, st, P, &launches);
+  launch(K.det, dim3(ctx->CD), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(256), ctx->budget_smem, st, P, &launches);
   launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(256), 0, st, P, &launches);
-  launch(K.sample, dim3(ctx->CS), dim3(256), ctx->sample_smem, st, P, &launches);
+  launch(K.sample, dim3(ctx->CS), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.combine_sample, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
   return finish(ctx, launches);
 }
@@ -528,7 +529,7 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.sel = reinterpret_cast<int*>(ctx->ordk);
   int launches = 0;
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
-  launch(K.dense, dim3(ctx->CD), dim3(256), ctx->gather_smem, st, P, &launches);
+  launch(K.dense, dim3(ctx->CD), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.combine_dense, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
   return finish(ctx, launches);
 }

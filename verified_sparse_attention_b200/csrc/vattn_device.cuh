@@ -15,6 +15,9 @@
 
 namespace vattn {
 
+// bit of the device error word: a bounded wait in a kernel ran out
+constexpr unsigned kDevTimeout = 4u;
+
 constexpr int kHist1 = 2048;  // bins of digit 1 (key bits 31..21)
 constexpr int kHist2 = 2048;  // bins of digit 2 (key bits 20..10)
 constexpr int kHist3 = 1024;  // bins of digit 3 (key bits 9..0)

@@ -787,32 +787,6 @@ __device__ __forceinline__ int tail_position(const int* topk, int k, int s1, int
   return s1 + rho + lo;
 }
 
-// Stage the sorted top-k list of unit u in shared memory when it fits.
-__device__ __forceinline__ const int* stage_topk(const DevParams& P, int u, const UnitInfo& inf,
-                                                 int* s_topk) {
-  const int* g = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
-  if (inf.k > kTopkSmem) return g;
-  for (int i = threadIdx.x; i < inf.k; i += blockDim.x) s_topk[i] = g[i];
-  __syncthreads();
-  return s_topk;
-}
-
-// Position of entry i of unit u's selected list (I_f first, then draws).
-__device__ __forceinline__ int item_position(const DevParams& P, int u, const UnitInfo& inf,
-                                             const int* topk, int i, bool whole_tail) {
-  if (i < inf.nI) return P.sel[static_cast<size_t>(u) * P.max_ctx + i];
-  const int t = i - inf.nI;
-  int rho;
-  if (whole_tail) {
-    rho = t;
-  } else {
-    const unsigned w = draw_word(P.seed, static_cast<unsigned>(u / P.Hkv),
-                                 static_cast<unsigned>(u % P.Hkv), static_cast<unsigned>(t));
-    rho = lemire(w, inf.ntail);
-  }
-  return tail_position(topk, inf.k, inf.s1, rho);
-}
-
 // ============================================================ gathers
 // One kernel template, three modes, each a persistent grid over a flattened
 // list of items. Items are grouped in slices, two per unit (u, part): part 0
@@ -823,63 +797,130 @@ __device__ __forceinline__ int item_position(const DevParams& P, int u, const Un
 // grows at every segment boundary).
 //   det:    part 0 = I_f (or all of I_f and the tail when the tail is no
 //           larger than the pilot); part 1 = the p pilot draws. True scores
-//           of every query head go to pscore; the unit's last CTA computes
-//           the budget; the grid's last CTA writes the sample prefix.
+//           of every query head go to pscore for the budget.
 //   sample: part 0 = the whole tail when the budget covers it; part 1 = the
-//           draws t in [p, b). The unit's last CTA merges its det and sample
-//           records and writes the output.
-//   dense:  part 0 = every position; the unit's last CTA writes the output.
-// Rows are staged by cp.async into a per-warp double buffer, so each warp
-// computes one chunk while the next chunk's rows are in flight.
+//           draws t in [p, b).
+//   dense:  part 0 = every position.
 constexpr int kModeDet = 0, kModeSample = 1, kModeDense = 2;
 
-// Row-per-lane-pair gather: each pair of lanes of a warp owns one gathered row
-// of a batch of 16 (even lane: even 16-byte chunks, odd lane: odd chunks; the
-// halving tree over chunks pairs chunks of equal parity until its last add).
-// K and V rows are staged in shared memory, XOR-swizzled by chunk so lanes
-// reading the same logical chunk of different rows hit different banks. Each
-// lane also owns D/32 output dimensions of the value accumulation.
+// Each warp streams its blocks of R rows through a private ring of NS
+// shared-memory stages: one lane per row issues two bulk copies (the K row
+// and the V row) that complete on the stage's mbarrier, NS - 1 blocks ahead
+// of the block being computed, so the bytes in flight live in shared memory
+// rather than registers. In a block, a row is NC = D / E lanes wide (one
+// 16-byte chunk each) and a warp step covers RPW = 32 / NC rows; UNR steps
+// make a block. Every lane computes its chunk's partial dot product for all
+// UNR rows and G heads (V = UNR * G values); one transposed reduction over
+// the NC lanes of a row then leaves each lane owning whole dot products (the
+// chunk sums are added pairwise at halving strides, the same tree as the
+// scoring order). The block's softmax weights go through shared memory to the
+// lanes that accumulate V.
 template <typename T, int D, int G>
 struct GatherShape {
   static constexpr int E = Elem<T>::kPer16;        // elements per 16-byte chunk
-  static constexpr int NC = D / E;                 // chunks per row
+  static constexpr int NC = D / E;                 // chunks (lanes) per row
   static constexpr int LOGNC = ilog2c(NC);
+  static constexpr int RPW = 32 / NC;              // rows per warp step
+  static constexpr int UNR = 4;                    // steps per block
+  static constexpr int R = RPW * UNR;              // rows per block
   static constexpr int ROWB = D * static_cast<int>(sizeof(T));
-  static constexpr int DPL = D / 32;               // value dims per lane
-  static constexpr int NW = 8;                     // warps per CTA
-  static constexpr int BATCH = 16;                 // items per warp batch (one per lane pair)
-  static constexpr int STAGE = BATCH * 2 * ROWB;   // K rows then V rows of a batch
+  static constexpr int BLKB = 2 * R * ROWB;        // K rows, then V rows (4 KB)
+  static constexpr int NW = G >= 8 ? 8 : 12;       // warps per CTA
+  static constexpr int NS = G >= 8 ? 6 : 4;        // ring stages per warp
+  static constexpr int V = UNR * G;                // partial dot products per lane
+  static constexpr int LOGV = ilog2c(V);
+  static constexpr int NVF = LOGV >= LOGNC ? (V >> LOGNC) : 1;             // owned per lane
+  static constexpr int REP = LOGV >= LOGNC ? 1 : (1 << (LOGNC - LOGV));    // lanes per score
   static constexpr int REC = G * (2 + D);          // floats per record: (m, l, acc[D]) per head
-  static constexpr size_t RED = static_cast<size_t>(NW) * G * D * 4;  // merge buffer (aliases the stages)
-  static constexpr size_t OFF_Q = (static_cast<size_t>(NW) * STAGE > RED ? static_cast<size_t>(NW) * STAGE : RED);
-  static constexpr size_t OFF_STAT = OFF_Q + static_cast<size_t>(G) * D * 4;  // [NW][G][2]
-  // dynamic shared memory; the sample gather appends its slice prefix
-  static constexpr size_t SMEM = OFF_STAT + static_cast<size_t>(NW) * G * 2 * 4;
+  static constexpr int WSP = 2 * R * G + 2 * G;    // per-warp floats: scores, weights, (m, cf)
+  static constexpr size_t RING = static_cast<size_t>(NW) * NS * BLKB;
+  static constexpr size_t RED = static_cast<size_t>(NW) * G * D * 4;    // merge buffer (aliases the rings)
+  static constexpr size_t OFF_Q = RING > RED ? RING : RED;
+  static constexpr size_t OFF_SP = OFF_Q + static_cast<size_t>(G) * D * 4;
+  static constexpr size_t OFF_L = OFF_SP + static_cast<size_t>(NW) * WSP * 4;
+  static constexpr size_t OFF_STAT = OFF_L + static_cast<size_t>(NW) * 32 * NVF * 4;
+  static constexpr size_t OFF_BAR = OFF_STAT + static_cast<size_t>(NW) * G * 2 * 4;
+  static constexpr size_t SMEM = OFF_BAR + static_cast<size_t>(NW) * NS * 8;
+  static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(SMEM <= 227 * 1024, "gather shared memory");
 };
 
-// Byte offset of logical chunk c of row r in a swizzled batch area.
-template <int NC>
-__device__ __forceinline__ int swz(int r, int c) {
-  return (r * NC + (c ^ (r & (NC - 1)))) * 16;
+// exp(x - m) with m a running maximum (0 while m is still -inf).
+__device__ __forceinline__ float exp_rel(float x, float m) {
+  return m == -INFINITY ? 0.0f : __expf(x - m);
 }
 
-__host__ __device__ constexpr int bitrev_c(int x, int bits) {
-  return bits == 0 ? 0 : ((x & 1) << (bits - 1)) | bitrev_c(x >> 1, bits - 1);
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Makes barrier initialisation visible to the async proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Bounded wait for the completion of the barrier phase with parity `parity`;
+// false when the limit ran out (each try may itself suspend for a while).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  const unsigned a = smem_u32(bar);
+  for (int it = 0; it < (1 << 20); it++) {
+    unsigned done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// Orders this thread's earlier generic shared-memory accesses before later
+// async-proxy writes (a bulk copy into a stage that was just read).
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  const size_t g = __cvta_generic_to_global(src);
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(g), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-  const size_t g = __cvta_generic_to_global(gsrc);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(g) : "memory");
-}
-// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void l2_prefetch(const void* gsrc, int bytes) {
-  const size_t g = __cvta_generic_to_global(gsrc);  // the instruction takes a global-space address
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(g), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Transposed reduction of NV values per lane over the lanes that differ in
+// bits O, O/2, ..., 1 of the lane index: while a lane holds more than one
+// value it keeps one half (the upper half when its bit O is set) and adds the
+// partner's copy of that half; once it holds one value, the remaining levels
+// are plain butterflies. Every sum pairs the same two subtrees as the halving
+// tree over chunks.
+template <int NV, int O>
+struct TReduce {
+  __device__ static __forceinline__ void run(float* x, int lane) {
+    if constexpr (O >= 1) {
+      if constexpr (NV > 1) {
+        const bool hi = (lane & O) != 0;
+#pragma unroll
+        for (int i = 0; i < NV / 2; i++) {
+          const float send = hi ? x[i] : x[i + NV / 2];
+          const float keep = hi ? x[i + NV / 2] : x[i];
+          x[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, O));
+        }
+        TReduce<NV / 2, O / 2>::run(x, lane);
+      } else {
+        x[0] = __fadd_rn(x[0], __shfl_xor_sync(0xffffffffu, x[0], O));
+        TReduce<1, O / 2>::run(x, lane);
+      }
+    }
+  }
+};
 
 // CTA of C holding flattened item x of T (CTA c owns [c*T/C, (c+1)*T/C)).
 __device__ __forceinline__ int cta_of(long long x, long long T, int C) {
@@ -1231,33 +1272,34 @@ __device__ __forceinline__ int unit_segments(const long long* pre, int u, long l
 
 // ============================================================ k_gather
 template <typename T, int D, int G, int MODE>
-__global__ void __launch_bounds__(256, (G >= 8 ? 2 : 3)) k_gather(DevParams P) {
+__global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(DevParams P) {
   using S = GatherShape<T, D, G>;
-  constexpr int E = S::E, NC = S::NC, LOGNC = S::LOGNC, DPL = S::DPL, NW = S::NW;
-  constexpr int DB = DPL * static_cast<int>(sizeof(T));  // value bytes per lane (4, 8 or 16)
+  constexpr int E = S::E, NC = S::NC, LOGNC = S::LOGNC, RPW = S::RPW, UNR = S::UNR, R = S::R;
+  constexpr int ROWB = S::ROWB, NW = S::NW, NS = S::NS, V = S::V, LOGV = S::LOGV, NVF = S::NVF,
+                REP = S::REP, REC = S::REC;
   extern __shared__ __align__(128) unsigned char smem[];
-  float* s_q = reinterpret_cast<float*>(smem + S::OFF_Q);
-  float* s_red = reinterpret_cast<float*>(smem);  // aliases the stages during merges
-  float* s_stat = reinterpret_cast<float*>(smem + S::OFF_STAT);
-  __shared__ unsigned s_warp[32];
-  __shared__ long long s_carry;
-
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row = lane >> 1, par = lane & 1;  // my row in the batch, my chunk parity
+  const int grp = lane / NC, c = lane % NC;
+  float* s_q = reinterpret_cast<float*>(smem + S::OFF_Q);
+  float* s_sc = reinterpret_cast<float*>(smem + S::OFF_SP) + warp * S::WSP;  // [R][G] scores
+  float* s_p = s_sc + R * G;                                                  // [RPW][UNR][G] weights
+  float* s_mc = s_p + R * G;                                                  // [G] maxima, [G] factors
+  float* s_ll = reinterpret_cast<float*>(smem + S::OFF_L) + warp * 32 * NVF;
+  float* s_stat = reinterpret_cast<float*>(smem + S::OFF_STAT);
+  float* s_red = reinterpret_cast<float*>(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR) + warp * NS;
+  unsigned char* ring = smem + static_cast<size_t>(warp) * NS * S::BLKB;
+
+  if (lane < NS) mbar_init(&bars[lane], 1);
+  mbar_init_fence();
+  __syncthreads();
   grid_dependency_wait();
-  long long* pre = (MODE == kModeSample) ? P.pre_samp : P.pre_det;
+
+  const long long* pre = (MODE == kModeSample) ? P.pre_samp : P.pre_det;
   float* rec = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
-  const int C = gridDim.x, c = blockIdx.x;
-  if (MODE == kModeSample) {
-    // the sample slices follow from the budgets; every CTA derives the prefix
-    // (CTA 0's copy is the one later kernels read)
-    long long* dst = (c == 0) ? pre : reinterpret_cast<long long*>(smem + S::SMEM);
-    write_slice_prefix<kModeSample>(P, dst, s_warp, &s_carry);
-    __syncthreads();
-    pre = dst;
-  }
+  const int C = gridDim.x, cta = blockIdx.x;
   const long long Tt = pre[2 * P.units];
-  const long long beg = Tt * c / C, end = Tt * (c + 1) / C;
+  const long long beg = Tt * cta / C, end = Tt * (cta + 1) / C;
   long long cur = beg;
   int sidx = 0;
   if (beg < end) {
@@ -1270,8 +1312,8 @@ __global__ void __launch_bounds__(256, (G >= 8 ? 2 : 3)) k_gather(DevParams P) {
   }
   const T* kc = static_cast<const T*>(P.k);
   const T* vc = static_cast<const T*>(P.v);
-  unsigned char* kb_s = smem + warp * S::STAGE;          // this warp's K rows
-  unsigned char* vb_s = kb_s + S::BATCH * S::ROWB;       // and V rows
+  unsigned issued = 0;  // blocks this warp issued in earlier slices (stage and phase follow from it)
+  bool failed = false;
 
   while (cur < end) {
     while (pre[sidx + 1] <= cur) sidx++;
@@ -1291,196 +1333,223 @@ __global__ void __launch_bounds__(256, (G >= 8 ? 2 : 3)) k_gather(DevParams P) {
     }
     float* ps = (MODE == kModeDet && inf.mode == 2) ? P.pscore + static_cast<size_t>(u) * P.max_ctx * G
                                                      : nullptr;
-    // local item l of this slice -> (item index i in the unit's list, cache
-    // position); positions of sampled entries were written by k_draws / k_budget
-    auto position = [&](int l, int& i) -> int {
-      if (MODE == kModeDense) {
-        i = l;
-        return l;
-      }
-      if (MODE == kModeDet) i = part == 0 ? l : n_det + l;
-      else i = inf.nI + (whole_tail ? l : inf.p + l);
-      return sel[i];
+    // item index in the unit's list of local item x of this slice
+    auto item_of = [&](int x) -> int {
+      const int l = lb + x;
+      if (MODE == kModeDense) return l;
+      if (MODE == kModeDet) return part == 0 ? l : n_det + l;
+      return inf.nI + (whole_tail ? l : inf.p + l);
     };
 
-    // queries of the group, fp32, in shared memory
+    // queries of the group: fp32 in shared memory, then my chunk in registers
     __syncthreads();
     for (int x = threadIdx.x; x < G * D; x += blockDim.x)
       s_q[x] = Elem<T>::load(P.q, (static_cast<size_t>(b) * P.Hq + h * G) * D + x);
     __syncthreads();
+    float q[G][E];
+#pragma unroll
+    for (int g = 0; g < G; g++)
+#pragma unroll
+      for (int e = 0; e < E; e++) q[g][e] = s_q[g * D + c * E + e];
 
-    float m[G], l[G], acc[G][DPL];
+    float m_run = -INFINITY;  // lane g < G: running maximum of head g
+    float l_own[NVF];
+    float acc[G][E];
 #pragma unroll
-    for (int g = 0; g < G; g++) {
-      m[g] = -INFINITY;
-      l[g] = 0.0f;
+    for (int j = 0; j < NVF; j++) l_own[j] = 0.0f;
 #pragma unroll
-      for (int d = 0; d < DPL; d++) acc[g][d] = 0.0f;
-    }
+    for (int g = 0; g < G; g++)
+#pragma unroll
+      for (int e = 0; e < E; e++) acc[g][e] = 0.0f;
+
     const int nitems = valid ? le - lb : 0;
-    const int nbatch = (nitems + S::BATCH - 1) / S::BATCH;
-    auto prefetch_rows = [&](int kbn) {  // next batch's rows into L2
-      const int xn = kbn + row;
-      if (kbn < nitems && xn < nitems && par == 0) {
-        int i2;
-        const size_t o2 = row_off(P, b, h, position(lb + xn, i2), D);
-        l2_prefetch(kc + o2, S::ROWB);
-        l2_prefetch(vc + o2, S::ROWB);
+    const int nblk = (nitems + R - 1) / R;
+    // this warp's blocks: warp + t * NW (none once a wait has failed)
+    const int nbw = (!failed && warp < nblk) ? (nblk - warp + NW - 1) / NW : 0;
+    int nis = 0;  // blocks issued in this slice
+
+    // producer side: lane r < R owns row r of a block
+    auto pos_of = [&](int t) -> int {
+      const int x = (warp + t * NW) * R + lane;
+      if (t >= nbw || lane >= R || x >= nitems) return -1;
+      if (MODE == kModeDense) return lb + x;
+      return sel[item_of(x)];
+    };
+    auto pid_of = [&](int pos) -> int {
+      return pos < 0 ? 0 : P.page_table[static_cast<size_t>(b) * P.pps + page_slot(P, pos)];
+    };
+    auto issue = [&](int t, int pos, int pid) {
+      const unsigned g = issued + static_cast<unsigned>(t);
+      const int st = static_cast<int>(g % NS);
+      const int nvalid = min(R, nitems - (warp + t * NW) * R);
+      unsigned char* dst = ring + st * S::BLKB;
+      fence_proxy_async();
+      if (lane == 0) mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(nvalid * 2 * ROWB));
+      __syncwarp();
+      nis++;
+      if (lane < nvalid) {
+        const size_t off = ((static_cast<size_t>(pid) * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps)) * D;
+        bulk_copy_g2s(dst + lane * ROWB, kc + off, ROWB, &bars[st]);
+        bulk_copy_g2s(dst + (R + lane) * ROWB, vc + off, ROWB, &bars[st]);
       }
     };
 
-    for (int kbi = warp; kbi < nbatch; kbi += NW) {
-      const int kb = kbi * S::BATCH;
-      const int x = kb + row;
-      const bool ok = x < nitems;
-      int item = 0;
-      long long off = 0;
-      if (ok && par == 0) {
-        const int pos = position(lb + x, item);
-        off = static_cast<long long>(row_off(P, b, h, pos, D));
-      }
-      off = __shfl_sync(0xffffffffu, off, lane & ~1);
-      prefetch_rows(kb + NW * S::BATCH);
-      if (ok) {
-#pragma unroll
-        for (int jj = 0; jj < NC / 2; jj++) {
-          const int cc = 2 * jj + par;
-          cp_async16(kb_s + swz<NC>(row, cc), kc + static_cast<size_t>(off) + cc * E);
-          cp_async16(vb_s + swz<NC>(row, cc), vc + static_cast<size_t>(off) + cc * E);
-        }
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncwarp();
+    // fill the ring; the address pipeline then runs one and two blocks ahead
+    // of the issue (page ids for block t + NS - 1, positions for t + NS)
+#pragma unroll 1
+    for (int t = 0; t < NS - 1 && t < nbw; t++) {
+      const int pos = pos_of(t);
+      issue(t, pos, pid_of(pos));
+    }
+    int posA = pos_of(NS - 1);
+    int pidA = pid_of(posA);
+    int posB = pos_of(NS);
 
-      // true scores of my row: my parity's chunk sums in bit-reversed order,
-      // merged as a binary counter (exactly the halving tree's pairs), then
-      // the tree's last add with the partner lane's half
-      float sc[G];
-      {
-        float st[G][LOGNC];
+#pragma unroll 1
+    for (int t = 0; t < nbw; t++) {
+      if (t + NS - 1 < nbw && !failed) issue(t + NS - 1, posA, pidA);
+      posA = posB;
+      pidA = pid_of(posA);
+      posB = pos_of(t + NS + 1);
+
+      if (t >= nis) continue;  // never issued (only after a failed wait)
+      const unsigned g = issued + static_cast<unsigned>(t);
+      const int st = static_cast<int>(g % NS);
+      // every lane waits; the warp goes on only if all saw the copies land
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
+        if (!failed && lane == 0) atomicOr(P.err, static_cast<unsigned>(kDevTimeout));
+        failed = true;
+      }
+      if (failed) continue;
+      const unsigned char* kb = ring + st * S::BLKB;
+      const unsigned char* vb = kb + R * ROWB;
+      const int row0 = (warp + t * NW) * R;
+
+      // partial dot products of my chunk, all steps and heads
+      float sv[V];
 #pragma unroll
-        for (int ii = 0; ii < NC / 2; ii++) {
-          const int cc = 2 * bitrev_c(ii, LOGNC - 1) + par;
-          const uint4 kr = *reinterpret_cast<const uint4*>(kb_s + swz<NC>(row, cc));
-          float kx[E];
-          Elem<T>::unpack(kr, kx);
+      for (int k = 0; k < UNR; k++) {
+        const uint4 kr = *reinterpret_cast<const uint4*>(kb + (k * RPW + grp) * ROWB + c * 16);
+        float kx[E];
+        Elem<T>::unpack(kr, kx);
 #pragma unroll
-          for (int g = 0; g < G; g++) {
-            const float* qg = s_q + g * D + cc * E;
-            float a = 0.0f;
+        for (int gg = 0; gg < G; gg++) {
+          float a = 0.0f;
 #pragma unroll
-            for (int e = 0; e < E; e++) a = __fmaf_rn(qg[e], kx[e], a);
-            int lev = 0;
-#pragma unroll
-            for (int bit = 0; bit < LOGNC - 1; bit++) {
-              if (((ii >> bit) & 1) == 0) break;
-              a = __fadd_rn(st[g][lev], a);
-              lev++;
-            }
-            st[g][lev] = a;
-          }
-        }
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-          const float mine = st[g][LOGNC - 1];
-          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-          sc[g] = ok ? __fmul_rn(__fadd_rn(mine, other), P.scale) : -INFINITY;
+          for (int e = 0; e < E; e++) a = __fmaf_rn(q[gg][e], kx[e], a);
+          sv[k * G + gg] = a;
         }
       }
-      if (ps != nullptr && ok && par == 0) {
+      TReduce<V, NC / 2>::run(sv, lane);
+
+      // scores I own: value v = step * G + head
+      const bool primary = REP == 1 || (c & (REP - 1)) == 0;
+      float s_own[NVF];
 #pragma unroll
-        for (int g = 0; g < G; g++) ps[static_cast<size_t>(item) * G + g] = sc[g];
-      }
-      // online softmax over the batch (each row counted once, by its even lane)
-      float ew[G];
-#pragma unroll
-      for (int g = 0; g < G; g++) {
-        float bm = sc[g];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-        if (bm > m[g]) {
-          const float cc = __expf(m[g] - bm);  // 0 while m = -inf
-          l[g] *= cc;
-#pragma unroll
-          for (int d = 0; d < DPL; d++) acc[g][d] *= cc;
-          m[g] = bm;
+      for (int j = 0; j < NVF; j++) {
+        const int v = LOGV >= LOGNC ? c * NVF + j : (c >> (LOGNC - LOGV));
+        const int k = v / G, gg = v % G, r = k * RPW + grp;
+        const bool ok = row0 + r < nitems;
+        s_own[j] = ok ? __fmul_rn(sv[j], P.scale) : -INFINITY;
+        if (primary) {
+          s_sc[r * G + gg] = s_own[j];
+          if (ps != nullptr && ok) ps[static_cast<size_t>(item_of(row0 + r)) * G + gg] = s_own[j];
         }
-        ew[g] = ok ? __expf(sc[g] - m[g]) : 0.0f;
-        float es = par == 0 ? ew[g] : 0.0f;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) es += __shfl_xor_sync(0xffffffffu, es, o);
-        l[g] += es;
-      }
-      // value accumulation: lane owns dims [lane * DPL, (lane + 1) * DPL)
-      const int cnt = min(S::BATCH, nitems - kb);
-      const int vchunk = (lane * DB) >> 4, vin = (lane * DB) & 15;
-      for (int t = 0; t < cnt; t++) {
-        float et[G];
-#pragma unroll
-        for (int g = 0; g < G; g++) et[g] = __shfl_sync(0xffffffffu, ew[g], 2 * t);
-        const unsigned char* vp = vb_s + swz<NC>(t, vchunk) + vin;
-        float vx[DPL];
-        if (DB == 16) {
-          const uint4 w = *reinterpret_cast<const uint4*>(vp);
-          float tmp[E];
-          Elem<T>::unpack(w, tmp);
-#pragma unroll
-          for (int d = 0; d < DPL; d++) vx[d] = tmp[d];
-        } else if (DB == 8) {
-          const uint2 w = *reinterpret_cast<const uint2*>(vp);
-          if (sizeof(T) == 2) {
-            vx[0] = __uint_as_float(w.x << 16);
-            vx[1] = __uint_as_float(w.x & 0xFFFF0000u);
-            if (DPL > 2) {
-              vx[DPL > 2 ? 2 : 0] = __uint_as_float(w.y << 16);
-              vx[DPL > 3 ? 3 : 0] = __uint_as_float(w.y & 0xFFFF0000u);
-            }
-          } else {
-            vx[0] = __uint_as_float(w.x);
-            vx[DPL > 1 ? 1 : 0] = __uint_as_float(w.y);
-          }
-        } else {
-          const unsigned w = *reinterpret_cast<const unsigned*>(vp);
-          vx[0] = __uint_as_float(w << 16);
-          vx[DPL > 1 ? 1 : 0] = __uint_as_float(w & 0xFFFF0000u);
-        }
-#pragma unroll
-        for (int g = 0; g < G; g++)
-#pragma unroll
-          for (int d = 0; d < DPL; d++) acc[g][d] = fmaf(et[g], vx[d], acc[g][d]);
       }
       __syncwarp();
-    }
-
-    // ---- merge the CTA's warps into one record for (CTA, slice)
-    __syncthreads();  // every warp is done with its stage (aliased by s_red)
-    if (lane == 0) {
+      if (lane < G) {
+        float bm = -INFINITY;
 #pragma unroll
-      for (int g = 0; g < G; g++) {
-        s_stat[(warp * G + g) * 2] = m[g];
-        s_stat[(warp * G + g) * 2 + 1] = l[g];
+        for (int r = 0; r < R; r++) bm = fmaxf(bm, s_sc[r * G + lane]);
+        const float mn = fmaxf(m_run, bm);
+        s_mc[lane] = mn;
+        s_mc[G + lane] = exp_rel(m_run, mn);
+        m_run = mn;
       }
-    }
-    __syncthreads();
-    float* r = rec + static_cast<size_t>(c + sidx) * S::REC;
+      __syncwarp();
+      float cf[G];
+      bool resc = false;
 #pragma unroll
-    for (int g = 0; g < G; g++) {
+      for (int gg = 0; gg < G; gg++) {
+        cf[gg] = s_mc[G + gg];
+        resc |= cf[gg] != 1.0f;
+      }
+      if (resc) {  // the same for every lane
+#pragma unroll
+        for (int gg = 0; gg < G; gg++)
+#pragma unroll
+          for (int e = 0; e < E; e++) acc[gg][e] *= cf[gg];
+      }
+#pragma unroll
+      for (int j = 0; j < NVF; j++) {
+        const int v = LOGV >= LOGNC ? c * NVF + j : (c >> (LOGNC - LOGV));
+        const int k = v / G, gg = v % G;  // gg depends on the lane: read its (m, cf) from shared memory
+        const float pj = s_own[j] == -INFINITY ? 0.0f : __expf(s_own[j] - s_mc[gg]);
+        if (primary) {
+          l_own[j] = l_own[j] * s_mc[G + gg] + pj;
+          s_p[(grp * UNR + k) * G + gg] = pj;
+        }
+      }
+      __syncwarp();
+      // value accumulation: my chunk of each of my rows, every head
+#pragma unroll
+      for (int k = 0; k < UNR; k++) {
+        float pw[G];
+#pragma unroll
+        for (int gg = 0; gg < G; gg++) pw[gg] = s_p[(grp * UNR + k) * G + gg];
+        if (row0 + k * RPW + grp < nitems) {  // rows past the end hold stale bytes
+          const uint4 vr = *reinterpret_cast<const uint4*>(vb + (k * RPW + grp) * ROWB + c * 16);
+          float vx[E];
+          Elem<T>::unpack(vr, vx);
+#pragma unroll
+          for (int gg = 0; gg < G; gg++)
+#pragma unroll
+            for (int e = 0; e < E; e++) acc[gg][e] = fmaf(pw[gg], vx[e], acc[gg][e]);
+        }
+      }
+      __syncwarp();  // the stage and the score buffers are free again
+    }
+    issued += static_cast<unsigned>(nbw);
+
+    // ---- merge: row groups of the warp, then the warps into one record
+#pragma unroll
+    for (int o = NC; o < 32; o <<= 1)
+#pragma unroll
+      for (int gg = 0; gg < G; gg++)
+#pragma unroll
+        for (int e = 0; e < E; e++) acc[gg][e] += __shfl_xor_sync(0xffffffffu, acc[gg][e], o);
+#pragma unroll
+    for (int j = 0; j < NVF; j++) s_ll[lane * NVF + j] = l_own[j];
+    __syncwarp();
+    if (lane < G) {
+      float lsum = 0.0f;
+      for (int x = 0; x < 32 * NVF; x++) {
+        const int ln = x / NVF, j = x % NVF, cc = ln % NC;
+        const int v = LOGV >= LOGNC ? cc * NVF + j : (cc >> (LOGNC - LOGV));
+        if (v % G == lane) lsum += s_ll[x];
+      }
+      s_stat[(warp * G + lane) * 2] = m_run;
+      s_stat[(warp * G + lane) * 2 + 1] = lsum;
+    }
+    __syncthreads();  // stats written; every warp is done with its ring (s_red aliases it)
+    float* r = rec + static_cast<size_t>(cta + sidx) * REC;
+#pragma unroll
+    for (int gg = 0; gg < G; gg++) {
       float mb = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NW; w++) mb = fmaxf(mb, s_stat[(w * G + g) * 2]);
-      const float cw = (m[g] == -INFINITY) ? 0.0f : __expf(m[g] - mb);
+      for (int w = 0; w < NW; w++) mb = fmaxf(mb, s_stat[(w * G + gg) * 2]);
+      const float mw = s_stat[(warp * G + gg) * 2];
+      const float cw = exp_rel(mw, mb);
+      if (grp == 0) {
 #pragma unroll
-      for (int d = 0; d < DPL; d++) s_red[(warp * G + g) * D + lane * DPL + d] = acc[g][d] * cw;
+        for (int e = 0; e < E; e++) s_red[(warp * G + gg) * D + c * E + e] = acc[gg][e] * cw;
+      }
       if (threadIdx.x == 0) {
         float lb2 = 0.0f;
 #pragma unroll
-        for (int w = 0; w < NW; w++) {
-          const float mw = s_stat[(w * G + g) * 2];
-          lb2 += (mw == -INFINITY) ? 0.0f : s_stat[(w * G + g) * 2 + 1] * __expf(mw - mb);
-        }
-        r[g * (2 + D)] = mb;
-        r[g * (2 + D) + 1] = lb2;
+        for (int w = 0; w < NW; w++) lb2 += s_stat[(w * G + gg) * 2 + 1] * exp_rel(s_stat[(w * G + gg) * 2], mb);
+        r[gg * (2 + D)] = mb;
+        r[gg * (2 + D) + 1] = lb2;
       }
     }
     __syncthreads();
@@ -1545,6 +1614,13 @@ __global__ void __launch_bounds__(256) k_draws(DevParams P) {
       t0 = inf.p;
       t1 = inf.bsz;
     }
+  }
+  if (PHASE == 1 && blockIdx.x == 0 && blockIdx.y == 0) {
+    // slice prefix of the sample gather (every unit's budget is known now)
+    __shared__ unsigned s_warp[32];
+    __shared__ long long s_carry;
+    write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
+    __syncthreads();
   }
   const int n = t1 - t0;
   const int a = t0 + static_cast<int>(static_cast<long long>(n) * blockIdx.y / gridDim.y);
