@@ -22,12 +22,10 @@ struct vattn_ctx {
   int units_max = 0;
   int nseg = 0;
   int score_grid = 0;
-  int CD = 0, CS = 0;      // gather grid sizes (det/dense, sample)
+  int gather_grid = 0;     // CTAs of each gather launch
+  int CD = 0, CS = 0;      // record producers (warps) of the det/dense and sample gathers
   size_t gather_smem = 0;   // gathers (all modes)
   int gather_threads = 0;
-  size_t budget_smem = 0;
-  size_t combine_smem = 0;
-  int combine_scr = 0;      // floats
   size_t select_smem = 0;   // 0: the selection runs as four grid-wide passes
   int draw_splits = 1;
   size_t ws_bytes = 0;
@@ -79,6 +77,47 @@ double normal_upper_quantile(double delta) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The driver's tensor-map encoder, reached through the runtime (the library
+// does not link the driver library itself).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Row maps of the K and V caches for the gathers: a 2-D [rows][d] view with
+// rows = num_pages * Hkv * page_size, one-row boxes of all d columns.
+int encode_row_maps(const vattn_config& c, const void* k, const void* v, int num_pages, DevParams* P) {
+  const unsigned long long rows =
+      static_cast<unsigned long long>(num_pages) * c.num_kv_heads * static_cast<unsigned long long>(c.page_size);
+  if (rows > 0x7FFFFFFFull) return VATTN_EINVAL;  // row coordinates are 32-bit
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return VATTN_ECUDA;
+  const cuuint64_t esz = c.dtype == VATTN_BF16 ? 2 : 4;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c.head_dim), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(c.head_dim) * esz};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(c.head_dim), 1u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType dt =
+      c.dtype == VATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  for (int i = 0; i < 2; i++) {
+    const CUresult r = fn(i ? &P->tmv : &P->tmk, dt, 2, const_cast<void*>(i ? v : k), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return VATTN_ECUDA;
+  }
+  return VATTN_OK;
+}
 
 // ---------------------------------------------------------------- dispatch
 struct Kernels {
@@ -189,7 +228,6 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->rec_samp = ctx->rec_samp;
   P->CD = ctx->CD;
   P->CS = ctx->CS;
-  P->combine_scr = ctx->combine_scr;
   P->err = ctx->err;
 }
 
@@ -269,17 +307,9 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   int gocc = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, K.gather_threads, ctx->gather_smem);
   if (gocc < 1) gocc = 1;
-  ctx->CD = ctx->CS = gocc * ctx->num_sms;
-  // the combine stages (m, l) and a scale factor per (record, head), and a
-  // unit has at most CD + CS + 2 records; the budget stages record maxima
-  ctx->combine_scr = (3 * G + 2) * (ctx->CD + ctx->CS + 2) + 4 * G;
-  ctx->combine_smem = static_cast<size_t>(ctx->combine_scr) * sizeof(float);
-  ctx->budget_smem = std::max(static_cast<size_t>(ctx->CD + 2) * G * sizeof(float),
-                              static_cast<size_t>(vattn::kTopkSmem) * sizeof(int));
+  ctx->gather_grid = gocc * ctx->num_sms;
+  ctx->CD = ctx->CS = ctx->gather_grid * (K.gather_threads / 32);
   ctx->draw_splits = std::max(1, (2 * ctx->num_sms + static_cast<int>(U) - 1) / static_cast<int>(U));
-  for (auto fn : {K.combine_sample, K.combine_dense})
-    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->combine_smem));
-  cudaFuncSetAttribute(K.budget, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->budget_smem));
   if (cudaGetLastError() != cudaSuccess) {
     delete ctx;
     return VATTN_ECUDA;
@@ -438,6 +468,7 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.z = ctx->cached_z;
   P.seed = prm->seed;
   P.num_pages = prm->num_pages;
+  if (const int rc = encode_row_maps(c, k_cache, v_cache, prm->num_pages, &P)) return ctx->last_status = rc;
   P.q = q;
   P.k = k_cache;
   P.v = v_cache;
@@ -483,11 +514,11 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
   }
   launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
-  launch(K.det, dim3(ctx->CD), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
-  launch(K.budget, dim3(P.units), dim3(256), ctx->budget_smem, st, P, &launches);
+  launch(K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  launch(K.budget, dim3(P.units), dim3(256), 0, st, P, &launches);
   launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(256), 0, st, P, &launches);
-  launch(K.sample, dim3(ctx->CS), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
-  launch(K.combine_sample, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
+  launch(K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  launch(K.combine_sample, dim3(P.units), dim3(ctx->G * c.head_dim), 0, st, P, &launches);
   return finish(ctx, launches);
 }
 
@@ -516,6 +547,7 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.pilot_min = 2;
   P.eps = 1.0f;
   P.num_pages = num_pages;
+  if (const int rc = encode_row_maps(c, k_cache, v_cache, num_pages, &P)) return ctx->last_status = rc;
   P.proxy = VATTN_EXACT;
   P.q = q;
   P.k = k_cache;
@@ -529,8 +561,8 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.sel = reinterpret_cast<int*>(ctx->ordk);
   int launches = 0;
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
-  launch(K.dense, dim3(ctx->CD), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
-  launch(K.combine_dense, dim3(P.units), dim3(256), ctx->combine_smem, st, P, &launches);
+  launch(K.dense, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  launch(K.combine_dense, dim3(P.units), dim3(ctx->G * c.head_dim), 0, st, P, &launches);
   return finish(ctx, launches);
 }
 

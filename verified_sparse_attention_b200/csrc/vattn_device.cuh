@@ -9,6 +9,7 @@
 // for the order it fixes.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -45,6 +46,9 @@ struct UnitInfo {
 };
 
 struct DevParams {
+  // 2-D row maps of the K and V caches ([rows][D], one-row boxes) for the
+  // row-gathering tensor copies; rows = num_pages * Hkv * page_size
+  CUtensorMap tmk, tmv;
   // shapes
   int Hq, Hkv, G, D;
   int pps;        // page-table entries per sequence
@@ -59,7 +63,6 @@ struct DevParams {
   unsigned long long seed;
   int nseg, dense;
   int CD, CS;       // grid sizes of the det (and dense) and sample gathers
-  int combine_scr;  // floats of shared scratch in k_combine
   // inputs
   const void* q;
   const void* k;

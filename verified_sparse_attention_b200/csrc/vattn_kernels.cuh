@@ -821,25 +821,22 @@ struct GatherShape {
   static constexpr int NC = D / E;                 // chunks (lanes) per row
   static constexpr int LOGNC = ilog2c(NC);
   static constexpr int RPW = 32 / NC;              // rows per warp step
-  static constexpr int UNR = 4;                    // steps per block
+  static constexpr int UNR = G >= 8 ? 4 : 8;       // steps per block
   static constexpr int R = RPW * UNR;              // rows per block
   static constexpr int ROWB = D * static_cast<int>(sizeof(T));
-  static constexpr int BLKB = 2 * R * ROWB;        // K rows, then V rows (4 KB)
-  static constexpr int NW = G >= 8 ? 8 : 12;       // warps per CTA
-  static constexpr int NS = G >= 8 ? 6 : 4;        // ring stages per warp
+  static constexpr int BLKB = 2 * R * ROWB;        // K rows, then V rows (4 or 8 KB)
+  static constexpr int NW = 8;                     // warps per CTA
+  static constexpr int NS = (192 * 1024) / (NW * BLKB);  // stages filling a 192 KB ring
   static constexpr int V = UNR * G;                // partial dot products per lane
   static constexpr int LOGV = ilog2c(V);
   static constexpr int NVF = LOGV >= LOGNC ? (V >> LOGNC) : 1;             // owned per lane
   static constexpr int REP = LOGV >= LOGNC ? 1 : (1 << (LOGNC - LOGV));    // lanes per score
   static constexpr int REC = G * (2 + D);          // floats per record: (m, l, acc[D]) per head
-  static constexpr int WSP = 2 * R * G + 2 * G;    // per-warp floats: scores, weights, (m, cf)
+  static constexpr int WSP = 3 * R * G + 2 * G;    // per-warp floats: scores, weight pairs, (m, cf)
   static constexpr size_t RING = static_cast<size_t>(NW) * NS * BLKB;
-  static constexpr size_t RED = static_cast<size_t>(NW) * G * D * 4;    // merge buffer (aliases the rings)
-  static constexpr size_t OFF_Q = RING > RED ? RING : RED;
-  static constexpr size_t OFF_SP = OFF_Q + static_cast<size_t>(G) * D * 4;
+  static constexpr size_t OFF_SP = RING;
   static constexpr size_t OFF_L = OFF_SP + static_cast<size_t>(NW) * WSP * 4;
-  static constexpr size_t OFF_STAT = OFF_L + static_cast<size_t>(NW) * 32 * NVF * 4;
-  static constexpr size_t OFF_BAR = OFF_STAT + static_cast<size_t>(NW) * G * 2 * 4;
+  static constexpr size_t OFF_BAR = OFF_L + static_cast<size_t>(NW) * 32 * NVF * 4;
   static constexpr size_t SMEM = OFF_BAR + static_cast<size_t>(NW) * NS * 8;
   static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(SMEM <= 227 * 1024, "gather shared memory");
@@ -892,6 +889,18 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsign
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
       "l"(g), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Tensor copy of four rows (row indices y0..y3, all columns of a one-row
+// box) of the 2-D row map `map` into consecutive rows at dst, completing on
+// `bar`.
+__device__ __forceinline__ void gather4_g2s(void* dst, const CUtensorMap* map, int y0, int y1, int y2, int y3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
 
@@ -1141,138 +1150,109 @@ __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, cons
   __syncthreads();
 }
 
-// Max score per head over unit u's det records (both parts) into s_mh. The
-// record maxima are loaded by all threads at once, then reduced.
+// Max score per head over unit u's det records (both parts) into s_mh.
+// Thread x always reads head x % G (the block size is a multiple of G); the
+// per-thread maxima are then reduced per head.
 template <int D, int G>
-__device__ void det_record_max(const DevParams& P, int u, float* s_mh, float* s_scr) {
+__device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
   constexpr int REC = G * (2 + D);
+  __shared__ float s_w[32][G];
   const long long T = P.pre_det[2 * P.units];
   int cf0, cl0, cf1, cl1;
   slice_ctas(P.pre_det, 2 * u, T, P.CD, cf0, cl0);
   slice_ctas(P.pre_det, 2 * u + 1, T, P.CD, cf1, cl1);
   const int n0 = max(0, cl0 - cf0 + 1), n1 = max(0, cl1 - cf1 + 1);
+  float m = -INFINITY;
   for (int x = threadIdx.x; x < (n0 + n1) * G; x += blockDim.x) {
     const int r = x / G, g = x % G;
     const size_t id = r < n0 ? static_cast<size_t>(cf0 + r + 2 * u) : static_cast<size_t>(cf1 + (r - n0) + 2 * u + 1);
-    s_scr[x] = P.rec_det[id * REC + g * (2 + D)];
+    m = fmaxf(m, P.rec_det[id * REC + g * (2 + D)]);
   }
+#pragma unroll
+  for (int o = 16; o >= G; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane < G) s_w[warp][lane] = m;
   __syncthreads();
   if (threadIdx.x < G) {
-    float m = -INFINITY;
-    for (int r = 0; r < n0 + n1; r++) m = fmaxf(m, s_scr[r * G + threadIdx.x]);
-    s_mh[threadIdx.x] = m;
+    float mm = -INFINITY;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); w++) mm = fmaxf(mm, s_w[w][threadIdx.x]);
+    s_mh[threadIdx.x] = mm;
   }
   __syncthreads();
 }
 
 // out = (A_0 + w A_1) / (L_0 + w L_1) for unit u from its records, with part 1
-// weighted by w = N_tail / b when the tail was sampled (1 otherwise). Block of
-// 256 threads; s_scr holds SCR floats (P.combine_scr when SCR is 0). A flat
-// table of the unit's records is built first; every record's (m, l) is then
-// loaded by all threads at once; maxima and scale factors come from shared
-// memory, and each output element sums its records' accumulators.
-template <int D, int G, int MODE, int SCR>
-__device__ void unit_combine(const DevParams& P, int u, float* s_scr) {
+// weighted by w = N_tail / b when the tail was sampled (1 otherwise). One
+// thread per (head, dimension) folds the records of each part in order with
+// a running maximum (the record loads do not depend on the fold, so they run
+// ahead of it).
+template <int D, int G, int MODE>
+__device__ void unit_combine(const DevParams& P, int u) {
   constexpr int REC = G * (2 + D);
-  __shared__ int s_tot;
   const UnitInfo inf = P.info[u];
   const int b = u / P.Hkv, h = u % P.Hkv;
+  const int g = threadIdx.x / D, e = threadIdx.x % D;
   const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
   const bool sampled = MODE == kModeSample && inf.mode == 2 && !inf.exhausted;
-  const int scr = SCR > 0 ? SCR : P.combine_scr;
-  // scratch layout: record table [tot] (offset in floats, part in the low bit
-  // of a separate int array), then (m, l) [tot][G][2], scale factors [tot][G],
-  // and M, L [2][G] at the end
-  long long* s_roff = reinterpret_cast<long long*>(s_scr);
-  float* s_M = s_scr + scr - 4 * G;
-  float* s_L = s_M + 2 * G;
-  if (threadIdx.x == 0) {
-    int tot = 0;
-    const long long Tm = (MODE == kModeSample) ? P.pre_samp[2 * P.units] : P.pre_det[2 * P.units];
-    const long long Td = P.pre_det[2 * P.units];
-    for (int part = 0; part < 2; part++) {
+  float M[2], L[2], A[2];
+#pragma unroll
+  for (int part = 0; part < 2; part++) {
+    float m = -INFINITY, l = 0.0f, a = 0.0f;
+    auto fold = [&](const long long* pre, const float* rec, int C) {
       int cf, cl;
-      // this kernel's records (the sample gather's, or the dense/det gather's)
-      slice_ctas(MODE == kModeSample ? P.pre_samp : P.pre_det, 2 * u + part, Tm,
-                 MODE == kModeSample ? P.CS : P.CD, cf, cl);
-      const float* base = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
-      const long long bo = base == P.rec_det ? 0 : (P.rec_samp - P.rec_det);
-      for (int c = cf; c <= cl; c++) s_roff[tot++] = ((bo + static_cast<long long>(c + 2 * u + part) * REC) << 1) | part;
-      // the det gather's records, in sample mode (the pilot is dropped when the
-      // whole tail is taken)
-      if (MODE == kModeSample && !(part == 1 && whole_tail)) {
-        slice_ctas(P.pre_det, 2 * u + part, Td, P.CD, cf, cl);
-        for (int c = cf; c <= cl; c++) s_roff[tot++] = (static_cast<long long>(c + 2 * u + part) * REC) << 1 | part;
+      slice_ctas(pre, 2 * u + part, pre[2 * P.units], C, cf, cl);
+      constexpr int B = 8;  // records loaded together, then folded
+      for (int c0 = cf; c0 <= cl; c0 += B) {
+        float rm[B], rl[B], ra[B];
+#pragma unroll
+        for (int j = 0; j < B; j++) {
+          rm[j] = -INFINITY;
+          rl[j] = ra[j] = 0.0f;
+          if (c0 + j <= cl) {
+            const float* r = rec + static_cast<size_t>(c0 + j + 2 * u + part) * REC + g * (2 + D);
+            rm[j] = r[0];
+            rl[j] = r[1];
+            ra[j] = r[2 + e];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < B; j++) {  // an empty record has m = -inf, l = 0, acc = 0
+          const float nm = fmaxf(m, rm[j]);
+          const float so = exp_rel(m, nm), sn = exp_rel(rm[j], nm);
+          l = l * so + rl[j] * sn;
+          a = a * so + ra[j] * sn;
+          m = nm;
+        }
       }
+    };
+    if (MODE == kModeSample) {
+      fold(P.pre_samp, P.rec_samp, P.CS);
+      // the det gather's records too (the pilot is dropped when the whole
+      // tail is taken)
+      if (!(part == 1 && whole_tail)) fold(P.pre_det, P.rec_det, P.CD);
+    } else {
+      fold(P.pre_det, P.rec_det, P.CD);
     }
-    s_tot = tot;
+    M[part] = m;
+    L[part] = l;
+    A[part] = a;
   }
-  __syncthreads();
-  const int tot = s_tot;
-  float* s_ml = s_scr + 2 * tot;          // after the table (tot long longs)
-  float* s_cf = s_ml + 2 * tot * G;
-  for (int x = threadIdx.x; x < tot * G * 2; x += blockDim.x) {
-    const int r = x / (2 * G), g = (x / 2) % G, f = x & 1;
-    s_ml[x] = P.rec_det[(s_roff[r] >> 1) + g * (2 + D) + f];
-  }
-  __syncthreads();
-  if (threadIdx.x < 2 * G) {
-    const int part = threadIdx.x / G, g = threadIdx.x % G;
-    float M = -INFINITY;
-    for (int r = 0; r < tot; r++)
-      if ((s_roff[r] & 1) == part) M = fmaxf(M, s_ml[(r * G + g) * 2]);
-    float Lsum = 0.0f;
-    for (int r = 0; r < tot; r++) {
-      if ((s_roff[r] & 1) != part) continue;
-      const float mr = s_ml[(r * G + g) * 2];
-      const float c = (mr == -INFINITY) ? 0.0f : __expf(mr - M);
-      s_cf[r * G + g] = c;
-      Lsum += s_ml[(r * G + g) * 2 + 1] * c;
-    }
-    s_M[part * G + g] = M;
-    s_L[part * G + g] = Lsum;
-  }
-  __syncthreads();
   float w = 1.0f;
   if (sampled) w = static_cast<float>(static_cast<double>(inf.ntail) / static_cast<double>(inf.bsz));
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int g = idx / D, e = idx % D;
-    float* out = P.out + (static_cast<size_t>(b) * P.Hq + h * G + g) * D + e;
-    if (inf.n <= 0) {
-      *out = 0.0f;
-      continue;
-    }
-    float A0 = 0.0f, A1 = 0.0f;
-#pragma unroll 4
-    for (int r = 0; r < tot; r++) {
-      const long long ro = s_roff[r];
-      const float c = s_cf[r * G + g];
-      const float v = (c != 0.0f) ? P.rec_det[(ro >> 1) + g * (2 + D) + 2 + e] * c : 0.0f;
-      if (ro & 1) A1 += v; else A0 += v;
-    }
-    const float M0 = s_M[g], M1 = s_M[G + g];
-    const float M = fmaxf(M0, M1);
-    const float c0 = (M0 == -INFINITY) ? 0.0f : __expf(M0 - M);
-    const float c1 = (M1 == -INFINITY) ? 0.0f : __expf(M1 - M);
-    *out = (A0 * c0 + w * (A1 * c1)) / (s_L[g] * c0 + w * (s_L[G + g] * c1));
+  float* out = P.out + (static_cast<size_t>(b) * P.Hq + h * G + g) * D + e;
+  if (inf.n <= 0) {
+    *out = 0.0f;
+    return;
   }
-  __syncthreads();
+  const float Mx = fmaxf(M[0], M[1]);
+  const float c0 = exp_rel(M[0], Mx), c1 = exp_rel(M[1], Mx);
+  *out = (A[0] * c0 + w * (A[1] * c1)) / (L[0] * c0 + w * (L[1] * c1));
 }
 
-// Number of (CTA, slice) segments of unit u in this kernel.
-__device__ __forceinline__ int unit_segments(const long long* pre, int u, long long T, int C) {
-  int n = 0;
-  for (int part = 0; part < 2; part++) {
-    int cf, cl;
-    slice_ctas(pre, 2 * u + part, T, C, cf, cl);
-    n += max(0, cl - cf + 1);
-  }
-  return n;
-}
 
 // ============================================================ k_gather
 template <typename T, int D, int G, int MODE>
-__global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(DevParams P) {
+__global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(const __grid_constant__ DevParams P) {
   using S = GatherShape<T, D, G>;
   constexpr int E = S::E, NC = S::NC, LOGNC = S::LOGNC, RPW = S::RPW, UNR = S::UNR, R = S::R;
   constexpr int ROWB = S::ROWB, NW = S::NW, NS = S::NS, V = S::V, LOGV = S::LOGV, NVF = S::NVF,
@@ -1280,48 +1260,68 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / NC, c = lane % NC;
-  float* s_q = reinterpret_cast<float*>(smem + S::OFF_Q);
   float* s_sc = reinterpret_cast<float*>(smem + S::OFF_SP) + warp * S::WSP;  // [R][G] scores
-  float* s_p = s_sc + R * G;                                                  // [RPW][UNR][G] weights
-  float* s_mc = s_p + R * G;                                                  // [G] maxima, [G] factors
+  float* s_p = s_sc + R * G;                          // [RPW][UNR][G] weights, each stored twice (a pair)
+  float* s_mc = s_p + 2 * R * G;                      // [G] maxima, [G] factors
   float* s_ll = reinterpret_cast<float*>(smem + S::OFF_L) + warp * 32 * NVF;
-  float* s_stat = reinterpret_cast<float*>(smem + S::OFF_STAT);
-  float* s_red = reinterpret_cast<float*>(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR) + warp * NS;
   unsigned char* ring = smem + static_cast<size_t>(warp) * NS * S::BLKB;
 
+  __shared__ int s_first;
   if (lane < NS) mbar_init(&bars[lane], 1);
+  if (threadIdx.x == 0) s_first = 0;
   mbar_init_fence();
   __syncthreads();
   grid_dependency_wait();
 
+  // every warp is a record producer: warp gw of W owns items [T*gw/W, T*(gw+1)/W)
   const long long* pre = (MODE == kModeSample) ? P.pre_samp : P.pre_det;
   float* rec = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
-  const int C = gridDim.x, cta = blockIdx.x;
+  const int W = gridDim.x * NW, gw = blockIdx.x * NW + warp;
   const long long Tt = pre[2 * P.units];
-  const long long beg = Tt * cta / C, end = Tt * (cta + 1) / C;
-  long long cur = beg;
-  int sidx = 0;
-  if (beg < end) {
-    int lo = 0, hi = 2 * P.units;  // largest s with pre[s] <= beg
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (pre[mid] <= beg) lo = mid; else hi = mid;
-    }
-    sidx = lo;
-  }
+  const long long cbeg = Tt * (blockIdx.x * NW) / W, cend = Tt * ((blockIdx.x + 1) * NW) / W;
+  // the CTA's first slice: the one non-empty slice holding item cbeg
+  if (cbeg < cend)
+    for (int s = threadIdx.x; s < 2 * P.units; s += blockDim.x)
+      if (pre[s] <= cbeg && cbeg < pre[s + 1]) s_first = s;
+  __syncthreads();
+  int sidx = s_first;
+  const long long wbeg = Tt * gw / W, wend = Tt * (gw + 1) / W;
+  long long cur = wbeg;
   const T* kc = static_cast<const T*>(P.k);
   const T* vc = static_cast<const T*>(P.v);
   unsigned issued = 0;  // blocks this warp issued in earlier slices (stage and phase follow from it)
   bool failed = false;
 
-  while (cur < end) {
+  while (cur < wend) {
     while (pre[sidx + 1] <= cur) sidx++;
-    const long long send = min(end, pre[sidx + 1]);
+    const long long send = min(wend, pre[sidx + 1]);
     const int u = sidx >> 1, part = sidx & 1;
     const int lb = static_cast<int>(cur - pre[sidx]), le = static_cast<int>(send - pre[sidx]);
-    const UnitInfo inf = P.info[u];
     const int b = u / P.Hkv, h = u % P.Hkv;
+    // my chunk of every head's query, the unit's state and, for a contiguous
+    // cache, its one page: all loads issued together
+    // packed FMAs compute two dot products at once, each half its own fp32
+    // chain: for G < 8 two rows (steps k, k + 1) of one head, with each query
+    // element stored twice; for G = 8 two heads of one row (fewer registers)
+    constexpr bool kPairSteps = G < 8;
+    constexpr int QP = kPairSteps ? G : G / 2;
+    float2 q2[QP][E];
+#pragma unroll
+    for (int j = 0; j < QP; j++)
+#pragma unroll
+      for (int e = 0; e < E; e++) {
+        const size_t qrow = static_cast<size_t>(b) * P.Hq + h * G;
+        if (kPairSteps) {
+          const float qv = Elem<T>::load(P.q, (qrow + j) * D + c * E + e);
+          q2[j][e] = make_float2(qv, qv);
+        } else {
+          q2[j][e] = make_float2(Elem<T>::load(P.q, (qrow + 2 * j) * D + c * E + e),
+                                 Elem<T>::load(P.q, (qrow + 2 * j + 1) * D + c * E + e));
+        }
+      }
+    const UnitInfo inf = P.info[u];
+    const int pid_c = P.pps == 1 ? P.page_table[static_cast<size_t>(b) * P.pps] : 0;
     const bool valid = inf.n > 0;
     const int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
     const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
@@ -1341,67 +1341,100 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
       return inf.nI + (whole_tail ? l : inf.p + l);
     };
 
-    // queries of the group: fp32 in shared memory, then my chunk in registers
-    __syncthreads();
-    for (int x = threadIdx.x; x < G * D; x += blockDim.x)
-      s_q[x] = Elem<T>::load(P.q, (static_cast<size_t>(b) * P.Hq + h * G) * D + x);
-    __syncthreads();
-    float q[G][E];
-#pragma unroll
-    for (int g = 0; g < G; g++)
-#pragma unroll
-      for (int e = 0; e < E; e++) q[g][e] = s_q[g * D + c * E + e];
-
     float m_run = -INFINITY;  // lane g < G: running maximum of head g
     float l_own[NVF];
-    float acc[G][E];
+    float2 acc[G][E / 2];
 #pragma unroll
     for (int j = 0; j < NVF; j++) l_own[j] = 0.0f;
 #pragma unroll
     for (int g = 0; g < G; g++)
 #pragma unroll
-      for (int e = 0; e < E; e++) acc[g][e] = 0.0f;
+      for (int e = 0; e < E / 2; e++) acc[g][e] = make_float2(0.0f, 0.0f);
 
     const int nitems = valid ? le - lb : 0;
     const int nblk = (nitems + R - 1) / R;
-    // this warp's blocks: warp + t * NW (none once a wait has failed)
-    const int nbw = (!failed && warp < nblk) ? (nblk - warp + NW - 1) / NW : 0;
+    // this warp's blocks of R consecutive items (none once a wait has failed)
+    const int nbw = failed ? 0 : nblk;
     int nis = 0;  // blocks issued in this slice
 
     // producer side: lane r < R owns row r of a block
     auto pos_of = [&](int t) -> int {
-      const int x = (warp + t * NW) * R + lane;
+      const int x = t * R + lane;
       if (t >= nbw || lane >= R || x >= nitems) return -1;
       if (MODE == kModeDense) return lb + x;
-      return sel[item_of(x)];
+      const int i = item_of(x);
+      if (MODE == kModeDet && part == 0) {  // sinks and window follow from the regions
+        if (i < inf.s1) return i;
+        if (i >= inf.s1 + inf.k && i < inf.nI) return inf.wst + (i - inf.s1 - inf.k);
+      }
+      return sel[i];
     };
     auto pid_of = [&](int pos) -> int {
+      if (P.pps == 1) return pid_c;
       return pos < 0 ? 0 : P.page_table[static_cast<size_t>(b) * P.pps + page_slot(P, pos)];
     };
     auto issue = [&](int t, int pos, int pid) {
       const unsigned g = issued + static_cast<unsigned>(t);
       const int st = static_cast<int>(g % NS);
-      const int nvalid = min(R, nitems - (warp + t * NW) * R);
+      const int nvalid = min(R, nitems - t * R);
       unsigned char* dst = ring + st * S::BLKB;
       fence_proxy_async();
-      if (lane == 0) mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(nvalid * 2 * ROWB));
-      __syncwarp();
       nis++;
-      if (lane < nvalid) {
-        const size_t off = ((static_cast<size_t>(pid) * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps)) * D;
-        bulk_copy_g2s(dst + lane * ROWB, kc + off, ROWB, &bars[st]);
-        bulk_copy_g2s(dst + (R + lane) * ROWB, vc + off, ROWB, &bars[st]);
+      // row index in the [rows][D] view of the caches; rows adjacent in
+      // memory form runs (a lane starts one when its row does not directly
+      // follow the previous lane's)
+      int row = lane < nvalid ? (pid * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps) : 0;
+      const int prev = __shfl_up_sync(0xffffffffu, row, 1);
+      const bool start = lane < nvalid && (lane == 0 || row != prev + 1);
+      const unsigned starts = __ballot_sync(0xffffffffu, start);
+      if (__popc(starts) <= R / 4) {
+        // few runs: one bulk copy per run; rows past the end get zero V so
+        // that their zero weights give exact zeros
+        if (lane == 0) mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(nvalid * 2 * ROWB));
+        __syncwarp();
+        if (start) {
+          const unsigned later = starts & ~((2u << lane) - 1u);  // run starts after mine
+          const int stop = later ? __ffs(later) - 1 : nvalid;
+          const unsigned bytes = static_cast<unsigned>((stop - lane) * ROWB);
+          const size_t off = static_cast<size_t>(row) * D;
+          bulk_copy_g2s(dst + lane * ROWB, kc + off, bytes, &bars[st]);
+          bulk_copy_g2s(dst + (R + lane) * ROWB, vc + off, bytes, &bars[st]);
+        } else if (lane >= nvalid && lane < R) {
+          uint4* z = reinterpret_cast<uint4*>(dst + (R + lane) * ROWB);
+#pragma unroll
+          for (int i = 0; i < ROWB / 16; i++) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+        // scattered rows: four per tensor copy; rows past the end repeat
+        // row 0 (finite values under zero weights)
+        const int row0v = __shfl_sync(0xffffffffu, row, 0);
+        if (lane >= nvalid) row = row0v;
+        const int r1 = __shfl_down_sync(0xffffffffu, row, 1);
+        const int r2 = __shfl_down_sync(0xffffffffu, row, 2);
+        const int r3 = __shfl_down_sync(0xffffffffu, row, 3);
+        if (lane == 0) mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(R * 2 * ROWB));
+        __syncwarp();
+        if (lane < R && (lane & 3) == 0) {
+          gather4_g2s(dst + lane * ROWB, &P.tmk, row, r1, r2, r3, &bars[st]);
+          gather4_g2s(dst + (R + lane) * ROWB, &P.tmv, row, r1, r2, r3, &bars[st]);
+        }
       }
     };
 
     // fill the ring; the address pipeline then runs one and two blocks ahead
     // of the issue (page ids for block t + NS - 1, positions for t + NS)
-#pragma unroll 1
-    for (int t = 0; t < NS - 1 && t < nbw; t++) {
-      const int pos = pos_of(t);
-      issue(t, pos, pid_of(pos));
+    int posA;
+    {
+      int posq[NS], pidq[NS - 1];  // loads of the first blocks, issued together
+#pragma unroll
+      for (int t = 0; t < NS; t++) posq[t] = pos_of(t);
+#pragma unroll
+      for (int t = 0; t < NS - 1; t++) pidq[t] = pid_of(posq[t]);
+#pragma unroll
+      for (int t = 0; t < NS - 1; t++)
+        if (t < nbw) issue(t, posq[t], pidq[t]);
+      posA = posq[NS - 1];
     }
-    int posA = pos_of(NS - 1);
     int pidA = pid_of(posA);
     int posB = pos_of(NS);
 
@@ -1423,21 +1456,41 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
       if (failed) continue;
       const unsigned char* kb = ring + st * S::BLKB;
       const unsigned char* vb = kb + R * ROWB;
-      const int row0 = (warp + t * NW) * R;
+      const int row0 = t * R;
 
       // partial dot products of my chunk, all steps and heads
       float sv[V];
+      if constexpr (kPairSteps) {
 #pragma unroll
-      for (int k = 0; k < UNR; k++) {
-        const uint4 kr = *reinterpret_cast<const uint4*>(kb + (k * RPW + grp) * ROWB + c * 16);
-        float kx[E];
-        Elem<T>::unpack(kr, kx);
+        for (int k = 0; k < UNR; k += 2) {
+          const uint4 kr0 = *reinterpret_cast<const uint4*>(kb + (k * RPW + grp) * ROWB + c * 16);
+          const uint4 kr1 = *reinterpret_cast<const uint4*>(kb + ((k + 1) * RPW + grp) * ROWB + c * 16);
+          float kx0[E], kx1[E];
+          Elem<T>::unpack(kr0, kx0);
+          Elem<T>::unpack(kr1, kx1);
 #pragma unroll
-        for (int gg = 0; gg < G; gg++) {
-          float a = 0.0f;
+          for (int gg = 0; gg < G; gg++) {
+            float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int e = 0; e < E; e++) a = __fmaf_rn(q[gg][e], kx[e], a);
-          sv[k * G + gg] = a;
+            for (int e = 0; e < E; e++) a = __ffma2_rn(q2[gg][e], make_float2(kx0[e], kx1[e]), a);
+            sv[k * G + gg] = a.x;
+            sv[(k + 1) * G + gg] = a.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < UNR; k++) {
+          const uint4 kr = *reinterpret_cast<const uint4*>(kb + (k * RPW + grp) * ROWB + c * 16);
+          float kx[E];
+          Elem<T>::unpack(kr, kx);
+#pragma unroll
+          for (int j = 0; j < QP; j++) {
+            float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int e = 0; e < E; e++) a = __ffma2_rn(q2[j][e], make_float2(kx[e], kx[e]), a);
+            sv[k * G + 2 * j] = a.x;
+            sv[k * G + 2 * j + 1] = a.y;
+          }
         }
       }
       TReduce<V, NC / 2>::run(sv, lane);
@@ -1478,7 +1531,10 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
 #pragma unroll
         for (int gg = 0; gg < G; gg++)
 #pragma unroll
-          for (int e = 0; e < E; e++) acc[gg][e] *= cf[gg];
+          for (int e = 0; e < E / 2; e++) {
+            acc[gg][e].x *= cf[gg];
+            acc[gg][e].y *= cf[gg];
+          }
       }
 #pragma unroll
       for (int j = 0; j < NVF; j++) {
@@ -1487,40 +1543,52 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
         const float pj = s_own[j] == -INFINITY ? 0.0f : __expf(s_own[j] - s_mc[gg]);
         if (primary) {
           l_own[j] = l_own[j] * s_mc[G + gg] + pj;
-          s_p[(grp * UNR + k) * G + gg] = pj;
+          reinterpret_cast<float2*>(s_p)[(grp * UNR + k) * G + gg] = make_float2(pj, pj);
         }
       }
       __syncwarp();
       // value accumulation: my chunk of each of my rows, every head
 #pragma unroll
       for (int k = 0; k < UNR; k++) {
-        float pw[G];
+        float2 pw[G];
+        const float2* pk = reinterpret_cast<const float2*>(s_p) + (grp * UNR + k) * G;
+        if constexpr (G % 2 == 0) {
 #pragma unroll
-        for (int gg = 0; gg < G; gg++) pw[gg] = s_p[(grp * UNR + k) * G + gg];
-        if (row0 + k * RPW + grp < nitems) {  // rows past the end hold stale bytes
-          const uint4 vr = *reinterpret_cast<const uint4*>(vb + (k * RPW + grp) * ROWB + c * 16);
-          float vx[E];
-          Elem<T>::unpack(vr, vx);
-#pragma unroll
-          for (int gg = 0; gg < G; gg++)
-#pragma unroll
-            for (int e = 0; e < E; e++) acc[gg][e] = fmaf(pw[gg], vx[e], acc[gg][e]);
+          for (int gg = 0; gg < G; gg += 2) {
+            const float4 w4 = *reinterpret_cast<const float4*>(pk + gg);
+            pw[gg] = make_float2(w4.x, w4.y);
+            pw[gg + 1] = make_float2(w4.z, w4.w);
+          }
+        } else {
+          pw[0] = pk[0];
         }
+        const uint4 vr = *reinterpret_cast<const uint4*>(vb + (k * RPW + grp) * ROWB + c * 16);
+        float vx[E];
+        Elem<T>::unpack(vr, vx);
+#pragma unroll
+        for (int gg = 0; gg < G; gg++)
+#pragma unroll
+          for (int e = 0; e < E / 2; e++)
+            acc[gg][e] = __ffma2_rn(pw[gg], make_float2(vx[2 * e], vx[2 * e + 1]), acc[gg][e]);
       }
       __syncwarp();  // the stage and the score buffers are free again
     }
     issued += static_cast<unsigned>(nbw);
 
-    // ---- merge: row groups of the warp, then the warps into one record
+    // ---- this warp's record for the slice: (m, l, acc[D]) per head
 #pragma unroll
     for (int o = NC; o < 32; o <<= 1)
 #pragma unroll
       for (int gg = 0; gg < G; gg++)
 #pragma unroll
-        for (int e = 0; e < E; e++) acc[gg][e] += __shfl_xor_sync(0xffffffffu, acc[gg][e], o);
+        for (int e = 0; e < E / 2; e++) {
+          acc[gg][e].x += __shfl_xor_sync(0xffffffffu, acc[gg][e].x, o);
+          acc[gg][e].y += __shfl_xor_sync(0xffffffffu, acc[gg][e].y, o);
+        }
 #pragma unroll
     for (int j = 0; j < NVF; j++) s_ll[lane * NVF + j] = l_own[j];
     __syncwarp();
+    float* r = rec + static_cast<size_t>(gw + sidx) * REC;
     if (lane < G) {
       float lsum = 0.0f;
       for (int x = 0; x < 32 * NVF; x++) {
@@ -1528,37 +1596,19 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(Dev
         const int v = LOGV >= LOGNC ? cc * NVF + j : (cc >> (LOGNC - LOGV));
         if (v % G == lane) lsum += s_ll[x];
       }
-      s_stat[(warp * G + lane) * 2] = m_run;
-      s_stat[(warp * G + lane) * 2 + 1] = lsum;
+      r[lane * (2 + D)] = m_run;
+      r[lane * (2 + D) + 1] = lsum;
     }
-    __syncthreads();  // stats written; every warp is done with its ring (s_red aliases it)
-    float* r = rec + static_cast<size_t>(cta + sidx) * REC;
+    if (grp == 0) {
 #pragma unroll
-    for (int gg = 0; gg < G; gg++) {
-      float mb = -INFINITY;
+      for (int gg = 0; gg < G; gg++)
 #pragma unroll
-      for (int w = 0; w < NW; w++) mb = fmaxf(mb, s_stat[(w * G + gg) * 2]);
-      const float mw = s_stat[(warp * G + gg) * 2];
-      const float cw = exp_rel(mw, mb);
-      if (grp == 0) {
-#pragma unroll
-        for (int e = 0; e < E; e++) s_red[(warp * G + gg) * D + c * E + e] = acc[gg][e] * cw;
-      }
-      if (threadIdx.x == 0) {
-        float lb2 = 0.0f;
-#pragma unroll
-        for (int w = 0; w < NW; w++) lb2 += s_stat[(w * G + gg) * 2 + 1] * exp_rel(s_stat[(w * G + gg) * 2], mb);
-        r[gg * (2 + D)] = mb;
-        r[gg * (2 + D) + 1] = lb2;
-      }
+        for (int e = 0; e < E / 2; e++) {
+          r[gg * (2 + D) + 2 + c * E + 2 * e] = acc[gg][e].x;
+          r[gg * (2 + D) + 2 + c * E + 2 * e + 1] = acc[gg][e].y;
+        }
     }
-    __syncthreads();
-    for (int x2 = threadIdx.x; x2 < G * D; x2 += blockDim.x) {
-      float a = 0.0f;
-#pragma unroll
-      for (int w = 0; w < NW; w++) a += s_red[w * G * D + x2];
-      r[(x2 / D) * (2 + D) + 2 + x2 % D] = a;
-    }
+    __syncwarp();  // s_ll is reused by the next slice
     cur = send;
   }
   grid_dependents_launch();
@@ -1635,22 +1685,21 @@ __global__ void __launch_bounds__(256) k_draws(DevParams P) {
 template <int D, int G>
 __global__ void __launch_bounds__(256) k_budget(DevParams P) {
   __shared__ float s_mh[G];
-  extern __shared__ __align__(128) unsigned char smem[];
   grid_dependency_wait();
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
-  if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh, reinterpret_cast<float*>(smem));
+  if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
   unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
   grid_dependents_launch();
 }
 
 // ============================================================ k_combine
-// One CTA per unit: merge its records and write the output.
+// One CTA per unit, one thread per (head, dimension): merge the unit's
+// records and write the output.
 template <int D, int G, int MODE>
-__global__ void __launch_bounds__(256) k_combine(DevParams P) {
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(G * D) k_combine(DevParams P) {
   grid_dependency_wait();
-  unit_combine<D, G, MODE, 0>(P, blockIdx.x, reinterpret_cast<float*>(smem));
+  unit_combine<D, G, MODE>(P, blockIdx.x);
   grid_dependents_launch();
 }
 
