@@ -26,7 +26,8 @@ struct vattn_ctx {
   int CD = 0, CS = 0;      // record producers (warps) of the det/dense and sample gathers
   size_t gather_smem = 0;   // gathers (all modes)
   int gather_threads = 0;
-  size_t select_smem = 0;   // 0: the selection runs as four grid-wide passes
+  bool select1 = false;     // one CTA per unit selects the top-k and draws the pilot
+  size_t select_smem = 0;   // else one cluster per unit (0: four grid-wide passes)
   int draw_splits = 1;
   size_t ws_bytes = 0;
   void* ws = nullptr;
@@ -358,8 +359,13 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
     delete ctx;
     return VATTN_ECUDA;
   }
-  // one cluster per unit selects the top-k when each CTA's key segment fits in
-  // shared memory; otherwise the four grid-wide passes do
+  // the top-k selection: one CTA per unit when the middle's keys fit in its
+  // shared memory, else one cluster per unit when each CTA's segment fits,
+  // else four grid-wide passes
+  ctx->select1 = cfg->max_ctx <= vattn::kSel1MaxKeys &&
+                 cudaFuncSetAttribute(vattn::k_select1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(vattn::kSel1Smem)) == cudaSuccess;
+  cudaGetLastError();
   {
     const size_t seg = (static_cast<size_t>(cfg->max_ctx) + vattn::kSelCluster - 1) / vattn::kSelCluster;
     const size_t bytes = vattn::kSelFixedSmem + seg * sizeof(unsigned);
@@ -505,15 +511,19 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     cudaEventRecord(ctx->ev_stop[ctx->ev_used], st);
     ctx->ev_used++;
   }
-  if (ctx->select_smem) {
-    launch(vattn::k_select, dim3(P.units * vattn::kSelCluster), dim3(256), ctx->select_smem, st, P, &launches);
+  if (ctx->select1) {
+    launch(vattn::k_select1, dim3(P.units), dim3(vattn::kSel1Threads), vattn::kSel1Smem, st, P, &launches);
   } else {
-    launch(vattn::k_sel_hist<2>, seg_grid, dim3(256), 0, st, P, &launches);
-    launch(vattn::k_sel_hist<3>, seg_grid, dim3(256), 0, st, P, &launches);
-    launch(vattn::k_sel_count, seg_grid, dim3(256), 0, st, P, &launches);
-    launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
+    if (ctx->select_smem) {
+      launch(vattn::k_select, dim3(P.units * vattn::kSelCluster), dim3(256), ctx->select_smem, st, P, &launches);
+    } else {
+      launch(vattn::k_sel_hist<2>, seg_grid, dim3(256), 0, st, P, &launches);
+      launch(vattn::k_sel_hist<3>, seg_grid, dim3(256), 0, st, P, &launches);
+      launch(vattn::k_sel_count, seg_grid, dim3(256), 0, st, P, &launches);
+      launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
+    }
+    launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
   }
-  launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
   launch(K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(256), 0, st, P, &launches);
   launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(256), 0, st, P, &launches);

@@ -352,4 +352,37 @@ __device__ __forceinline__ void find_digit(const unsigned* __restrict__ hist, in
   __syncthreads();
 }
 
+// find_digit for any block of BT threads over a shared-memory histogram
+// (each thread scans NB / BT consecutive bins downwards).
+template <int NB, int BT>
+__device__ __forceinline__ void find_digit_bt(const unsigned* hist, int krem, int* s_digit, int* s_krem,
+                                              unsigned* s_warp) {
+  constexpr int PER = NB / BT;
+  static_assert(PER >= 1 && NB % BT == 0, "bins per thread");
+  const int lo = NB - (threadIdx.x + 1) * PER;
+  unsigned v[PER];
+  unsigned sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    v[i] = hist[lo + i];
+    sum += v[i];
+  }
+  const unsigned incl = block_inclusive_scan(sum, s_warp);
+  const unsigned excl = incl - sum;
+  if (excl < static_cast<unsigned>(krem) && static_cast<unsigned>(krem) <= incl) {
+    unsigned c = excl;
+    bool done = false;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; i--) {
+      if (!done && c + v[i] >= static_cast<unsigned>(krem)) {
+        *s_digit = lo + i;
+        *s_krem = krem - static_cast<int>(c);
+        done = true;
+      }
+      c += v[i];
+    }
+  }
+  __syncthreads();
+}
+
 }  // namespace vattn

@@ -1637,6 +1637,190 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
   __syncthreads();
 }
 
+// ============================================================ k_select1
+// Top-k selection and pilot draws of one unit in one CTA of 1024 threads,
+// for middles of at most kSel1MaxKeys keys (staged in shared memory by one
+// bulk copy):
+//   digit 1 from the score pass's histogram; one pass over the keys builds
+//   the digit-2 histogram of the keys in bin d1 and collects their indices;
+//   digit 3 is counted over those candidates only (over all keys if they
+//   overflow kSel1Cand); one ordered pass writes the selected positions
+//   ascending (ties at the threshold to the lowest positions, as the key's
+//   low half orders them). The sorted list, kept in shared memory, then
+//   serves the pilot draws (or the whole tail when it is no larger than the
+//   pilot), as in k_draws<0>.
+constexpr int kSel1Threads = 1024;
+constexpr int kSel1MaxKeys = 45056;
+constexpr int kSel1Cand = kTopkSmem - kHist2;  // candidate slots; with the histogram, the top-k staging
+constexpr size_t kSel1Smem = static_cast<size_t>(kSel1MaxKeys + 4 + kTopkSmem) * 4;
+
+// Exclusive prefix over the 32 warps of a 1024-thread block of one value per
+// warp (v from lane 0); every thread gets its warp's prefix and the total.
+__device__ __forceinline__ unsigned warp_prefix_1024(unsigned v, unsigned* s_w, unsigned* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) s_w[warp] = v;
+  __syncthreads();
+  unsigned x = s_w[lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  *total = __shfl_sync(0xffffffffu, x, 31);
+  const unsigned excl = __shfl_sync(0xffffffffu, x, warp) - __shfl_sync(0xffffffffu, s_w[warp], 0);
+  __syncthreads();  // s_w may be reused
+  return excl;
+}
+
+__global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned* s_raw = reinterpret_cast<unsigned*>(smem);          // [kSel1MaxKeys + 4]
+  unsigned* s_hist = s_raw + kSel1MaxKeys + 4;                   // [kHist2], then
+  unsigned* s_cand = s_hist + kHist2;                            // [kSel1Cand]; both later the top-k
+  int* s_topk = reinterpret_cast<int*>(s_hist);
+  __shared__ unsigned s_warp[32];
+  __shared__ int s_digit, s_krem;
+  __shared__ unsigned s_ncand;
+  __shared__ __align__(8) uint64_t s_bar;
+  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) mbar_init(&s_bar, 1);
+  mbar_init_fence();
+  __syncthreads();
+  grid_dependency_wait();
+  const UnitInfo inf = P.info[u];
+  const int* topk = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;  // global copy
+  if (inf.k > 0) {
+    const int mlen = inf.wst - inf.s1;
+    const size_t kofs = static_cast<size_t>(u) * P.max_ctx + inf.s1;  // first key in ordk
+    const unsigned* ordk = P.ordk + kofs;
+    // keys at s_keys[0, mlen): s_keys sits at the source's offset within 16
+    // bytes, so the aligned middle of the range is one bulk copy
+    const int shift = static_cast<int>((reinterpret_cast<uintptr_t>(ordk) >> 2) & 3);
+    unsigned* s_keys = s_raw + shift;
+    const int head = min(mlen, (4 - shift) & 3);      // keys before the first 16-byte boundary
+    const int nbody = ((mlen - head) / 4) * 4;         // keys copied in bulk
+    if (tid == 0 && nbody > 0) {
+      mbar_arrive_expect_tx(&s_bar, static_cast<unsigned>(nbody) * 4u);
+      bulk_copy_g2s(s_keys + head, ordk + head, static_cast<unsigned>(nbody) * 4u, &s_bar);
+    }
+    if (tid < head) s_keys[tid] = ordk[tid];
+    if (tid < mlen - head - nbody) s_keys[head + nbody + tid] = ordk[head + nbody + tid];
+    const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHistAll;
+    for (int x = tid; x < kHist1; x += kSel1Threads) s_hist[x] = h1[x];
+    if (tid == 0) {
+      s_digit = 0;
+      s_krem = inf.k;
+      s_ncand = 0;
+    }
+    if (nbody > 0 && !__all_sync(0xffffffffu, mbar_wait(&s_bar, 0u)) && lane == 0)
+      atomicOr(P.err, kDevTimeout);
+    __syncthreads();
+    find_digit_bt<kHist1, kSel1Threads>(s_hist, inf.k, &s_digit, &s_krem, s_warp);
+    const unsigned d1 = static_cast<unsigned>(s_digit);
+    const int krem1 = s_krem;
+
+    // digit 2 over the keys of bin d1, collecting them
+    for (int x = tid; x < kHist2; x += kSel1Threads) s_hist[x] = 0u;
+    __syncthreads();
+    for (int x = tid; x < mlen; x += kSel1Threads) {
+      const unsigned o = s_keys[x];
+      if ((o >> 21) == d1) {
+        atomicAdd(&s_hist[(o >> 10) & 2047u], 1u);
+        const unsigned slot = atomicAdd(&s_ncand, 1u);
+        if (slot < static_cast<unsigned>(kSel1Cand)) s_cand[slot] = static_cast<unsigned>(x);
+      }
+    }
+    __syncthreads();
+    find_digit_bt<kHist2, kSel1Threads>(s_hist, krem1, &s_digit, &s_krem, s_warp);
+    const unsigned d2 = static_cast<unsigned>(s_digit);
+    const int krem2 = s_krem;
+    const unsigned ncand = s_ncand;
+
+    // digit 3 over the candidates of prefix (d1, d2)
+    const unsigned pre = d1 << 11 | d2;
+    for (int x = tid; x < kHist3; x += kSel1Threads) s_hist[x] = 0u;
+    __syncthreads();
+    if (ncand <= static_cast<unsigned>(kSel1Cand)) {
+      for (int i = tid; i < static_cast<int>(ncand); i += kSel1Threads) {
+        const unsigned o = s_keys[s_cand[i]];
+        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
+      }
+    } else {
+      for (int x = tid; x < mlen; x += kSel1Threads) {
+        const unsigned o = s_keys[x];
+        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
+      }
+    }
+    __syncthreads();
+    find_digit_bt<kHist3, kSel1Threads>(s_hist, krem2, &s_digit, &s_krem, s_warp);
+    const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
+    const unsigned need_eq = static_cast<unsigned>(s_krem);
+    if (tid == 0) {
+      P.info[u].thr = thr;
+      P.info[u].need_eq = static_cast<int>(need_eq);
+    }
+
+    // ordered compaction: warp w takes keys [base + 512 w, base + 512 (w + 1))
+    // lane-interleaved; ballots give the ranks in position order
+    int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+    const bool stage = inf.k <= kTopkSmem;
+    const unsigned lt = (1u << lane) - 1u;
+    unsigned taken = 0, eq_seen = 0;
+    constexpr int PER = 16;
+    for (int base = 0; base < mlen; base += PER * kSel1Threads) {
+      const int wb = base + warp * PER * 32;
+      unsigned keys[PER], eqm[PER];
+      unsigned neq = 0;
+#pragma unroll
+      for (int i = 0; i < PER; i++) {
+        const int x = wb + i * 32 + lane;
+        keys[i] = x < mlen ? s_keys[x] : 0u;
+        eqm[i] = __ballot_sync(0xffffffffu, x < mlen && keys[i] == thr);
+        neq += __popc(eqm[i]);
+      }
+      unsigned eq_tot, tk_tot;
+      unsigned eq_run = eq_seen + warp_prefix_1024(neq, s_warp, &eq_tot);
+      unsigned tkm[PER];
+      unsigned ntk = 0;
+#pragma unroll
+      for (int i = 0; i < PER; i++) {
+        const int x = wb + i * 32 + lane;
+        const bool e = (eqm[i] >> lane) & 1u;
+        const bool t = x < mlen && (keys[i] > thr || (e && eq_run + __popc(eqm[i] & lt) < need_eq));
+        tkm[i] = __ballot_sync(0xffffffffu, t);
+        ntk += __popc(tkm[i]);
+        eq_run += __popc(eqm[i]);
+      }
+      unsigned pos = taken + warp_prefix_1024(ntk, s_warp, &tk_tot);
+#pragma unroll
+      for (int i = 0; i < PER; i++) {
+        if ((tkm[i] >> lane) & 1u) {
+          const unsigned p = pos + __popc(tkm[i] & lt);
+          const int j = inf.s1 + wb + i * 32 + lane;
+          sel[p] = j;
+          if (stage) s_topk[p] = j;
+        }
+        pos += __popc(tkm[i]);
+      }
+      eq_seen += eq_tot;
+      taken += tk_tot;
+    }
+    __syncthreads();  // the staged list is complete
+    if (stage) topk = s_topk;
+  }
+
+  // pilot draws (mode 2), or the whole tail when it is no larger than the pilot (mode 1)
+  const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
+  const bool whole = inf.mode == 1;
+  int* dsel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
+  const unsigned bb = static_cast<unsigned>(u / P.Hkv), hh = static_cast<unsigned>(u % P.Hkv);
+  for (int t = tid; t < t1; t += kSel1Threads) {
+    const int rho = whole ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
+    dsel[t] = tail_position(topk, inf.k, inf.s1, rho);
+  }
+  grid_dependents_launch();
+}
+
 // ============================================================ k_draws
 // Positions of sampled entries, one thread per entry. PHASE 0 (before the det
 // gather): the p pilot draws, or the whole tail when it is no larger than the
