@@ -1654,24 +1654,6 @@ constexpr int kSel1MaxKeys = 45056;
 constexpr int kSel1Cand = kTopkSmem - kHist2;  // candidate slots; with the histogram, the top-k staging
 constexpr size_t kSel1Smem = static_cast<size_t>(kSel1MaxKeys + 4 + kTopkSmem) * 4;
 
-// Exclusive prefix over the 32 warps of a 1024-thread block of one value per
-// warp (v from lane 0); every thread gets its warp's prefix and the total.
-__device__ __forceinline__ unsigned warp_prefix_1024(unsigned v, unsigned* s_w, unsigned* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) s_w[warp] = v;
-  __syncthreads();
-  unsigned x = s_w[lane];
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  *total = __shfl_sync(0xffffffffu, x, 31);
-  const unsigned excl = __shfl_sync(0xffffffffu, x, warp) - __shfl_sync(0xffffffffu, s_w[warp], 0);
-  __syncthreads();  // s_w may be reused
-  return excl;
-}
-
 __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned* s_raw = reinterpret_cast<unsigned*>(smem);          // [kSel1MaxKeys + 4]
@@ -1760,50 +1742,56 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
       P.info[u].need_eq = static_cast<int>(need_eq);
     }
 
-    // ordered compaction: warp w takes keys [base + 512 w, base + 512 (w + 1))
-    // lane-interleaved; ballots give the ranks in position order
+    // ordered compaction through a bitmap: per round, warp w turns keys
+    // [base + 1024 w, base + 1024 (w + 1)) into 32 words (one pair of ballots
+    // per 32 keys; lane j keeps word j). Words follow position order across
+    // threads, so block scans give how many tied keys each word keeps (the
+    // lowest positions) and where its selections go.
     int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
     const bool stage = inf.k <= kTopkSmem;
-    const unsigned lt = (1u << lane) - 1u;
     unsigned taken = 0, eq_seen = 0;
-    constexpr int PER = 16;
-    for (int base = 0; base < mlen; base += PER * kSel1Threads) {
-      const int wb = base + warp * PER * 32;
-      unsigned keys[PER], eqm[PER];
-      unsigned neq = 0;
-#pragma unroll
-      for (int i = 0; i < PER; i++) {
-        const int x = wb + i * 32 + lane;
-        keys[i] = x < mlen ? s_keys[x] : 0u;
-        eqm[i] = __ballot_sync(0xffffffffu, x < mlen && keys[i] == thr);
-        neq += __popc(eqm[i]);
-      }
-      unsigned eq_tot, tk_tot;
-      unsigned eq_run = eq_seen + warp_prefix_1024(neq, s_warp, &eq_tot);
-      unsigned tkm[PER];
-      unsigned ntk = 0;
-#pragma unroll
-      for (int i = 0; i < PER; i++) {
-        const int x = wb + i * 32 + lane;
-        const bool e = (eqm[i] >> lane) & 1u;
-        const bool t = x < mlen && (keys[i] > thr || (e && eq_run + __popc(eqm[i] & lt) < need_eq));
-        tkm[i] = __ballot_sync(0xffffffffu, t);
-        ntk += __popc(tkm[i]);
-        eq_run += __popc(eqm[i]);
-      }
-      unsigned pos = taken + warp_prefix_1024(ntk, s_warp, &tk_tot);
-#pragma unroll
-      for (int i = 0; i < PER; i++) {
-        if ((tkm[i] >> lane) & 1u) {
-          const unsigned p = pos + __popc(tkm[i] & lt);
-          const int j = inf.s1 + wb + i * 32 + lane;
-          sel[p] = j;
-          if (stage) s_topk[p] = j;
+    __shared__ unsigned s_round[2];
+    for (int base = 0; base < mlen; base += 32 * kSel1Threads) {
+      const int wb = base + warp * 1024;
+      unsigned wgt = 0, weq = 0;
+#pragma unroll 8
+      for (int j = 0; j < 32; j++) {
+        const int x = wb + j * 32 + lane;
+        const unsigned o = x < mlen ? s_keys[x] : 0u;
+        const unsigned bg = __ballot_sync(0xffffffffu, x < mlen && o > thr);
+        const unsigned be = __ballot_sync(0xffffffffu, x < mlen && o == thr);
+        if (lane == j) {
+          wgt = bg;
+          weq = be;
         }
-        pos += __popc(tkm[i]);
       }
-      eq_seen += eq_tot;
-      taken += tk_tot;
+      const unsigned ne = __popc(weq);
+      const unsigned eq_incl = block_inclusive_scan(ne, s_warp);
+      const unsigned eq_before = eq_seen + eq_incl - ne;
+      const unsigned keep = need_eq > eq_before ? min(ne, need_eq - eq_before) : 0u;
+      unsigned wsel = wgt, e = weq;
+      for (unsigned c = 0; c < keep; c++) {  // the lowest `keep` tied positions
+        wsel |= e & (0u - e);
+        e &= e - 1u;
+      }
+      const unsigned nt = __popc(wsel);
+      const unsigned t_incl = block_inclusive_scan(nt, s_warp);
+      unsigned pos = taken + t_incl - nt;
+      while (wsel) {
+        const int j = inf.s1 + wb + lane * 32 + (__ffs(wsel) - 1);
+        sel[pos] = j;
+        if (stage) s_topk[pos] = j;
+        pos++;
+        wsel &= wsel - 1u;
+      }
+      if (tid == kSel1Threads - 1) {  // round totals: the last thread holds the inclusive sums
+        s_round[0] = eq_incl;
+        s_round[1] = t_incl;
+      }
+      __syncthreads();
+      eq_seen += s_round[0];
+      taken += s_round[1];
+      __syncthreads();
     }
     __syncthreads();  // the staged list is complete
     if (stage) topk = s_topk;
