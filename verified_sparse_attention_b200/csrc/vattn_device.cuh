@@ -223,9 +223,8 @@ __device__ __forceinline__ unsigned ord_key(float f) {
 // ---------------------------------------------------------------- Philox4x32-10
 // Salmon, Moraes, Dror, Shaw (SC'11). Draw t of unit (b, h) is word t%4 of the
 // block with counter (t/4, b, h, 0) under key (seed low, seed high).
-__device__ __forceinline__ unsigned draw_word(unsigned long long seed, unsigned b, unsigned h,
-                                              unsigned t) {
-  unsigned c0 = t >> 2, c1 = b, c2 = h, c3 = 0u;
+__device__ __forceinline__ uint4 draw_block(unsigned long long seed, unsigned b, unsigned h, unsigned blk) {
+  unsigned c0 = blk, c1 = b, c2 = h, c3 = 0u;
   unsigned k0 = static_cast<unsigned>(seed), k1 = static_cast<unsigned>(seed >> 32);
 #pragma unroll
   for (int round = 0; round < 10; round++) {
@@ -241,8 +240,13 @@ __device__ __forceinline__ unsigned draw_word(unsigned long long seed, unsigned 
     c2 = n2;
     c3 = lo0;
   }
+  return make_uint4(c0, c1, c2, c3);
+}
+__device__ __forceinline__ unsigned draw_word(unsigned long long seed, unsigned b, unsigned h,
+                                              unsigned t) {
+  const uint4 q = draw_block(seed, b, h, t >> 2);
   const unsigned w = t & 3u;
-  return w == 0 ? c0 : (w == 1 ? c1 : (w == 2 ? c2 : c3));
+  return w == 0 ? q.x : (w == 1 ? q.y : (w == 2 ? q.z : q.w));
 }
 
 // Lemire multiply-shift: a 32-bit uniform word onto [0, n).

@@ -966,7 +966,11 @@ __device__ void write_slice_prefix(const DevParams& P, long long* pre, unsigned*
     const int sidx = base + threadIdx.x;
     unsigned cnt = 0;
     if (sidx < ns) {
-      const UnitInfo inf = P.info[sidx >> 1];
+      UnitInfo inf;
+      const int4* src = reinterpret_cast<const int4*>(P.info + (sidx >> 1));
+      int4* dst = reinterpret_cast<int4*>(&inf);
+#pragma unroll
+      for (int i = 0; i < static_cast<int>(sizeof(UnitInfo) / 16); i++) dst[i] = __ldcg(src + i);
       int n0, n1;
       slice_counts<MODE>(inf, n0, n1);
       cnt = static_cast<unsigned>((sidx & 1) ? n1 : n0);
@@ -1026,12 +1030,12 @@ __device__ __forceinline__ U128 warp_sum_u128(U128 v) {
 // n_h = (z * N_tail * sigma / (eps * D))^2 with sigma^2 = (p S2 - S1^2) /
 // (p (p - 1)) and D = S_f + N_tail * S1 / p, in double in a fixed operation
 // order. b = max(p, max_h n_h); b >= N_tail takes the whole tail instead.
-// Block of 256 threads.
+// Block of up to 1024 threads.
 template <int G>
 __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, const float* ps,
                             const float* s_mh) {
-  __shared__ unsigned long long s_a[8][G], s_b[8][G];
-  __shared__ U128 s_c[8][G];
+  __shared__ unsigned long long s_a[32][G], s_b[32][G];
+  __shared__ U128 s_c[32][G];
   __shared__ int s_need[G];
   const int b = u / P.Hkv, h = u % P.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -1061,17 +1065,18 @@ __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, cons
     s2[g] = U128{0ull, 0ull};
   }
   constexpr int BATCH = 4;
-  for (int i0 = tid; i0 < nA; i0 += BATCH * 256) {
+  const int nt = blockDim.x;
+  for (int i0 = tid; i0 < nA; i0 += BATCH * nt) {
     float sv[BATCH][G];
 #pragma unroll
     for (int k = 0; k < BATCH; k++) {
-      const int i = i0 + k * 256;
+      const int i = i0 + k * nt;
 #pragma unroll
       for (int g = 0; g < G; g++) sv[k][g] = i < nA ? ps[static_cast<size_t>(i) * G + g] : 0.0f;
     }
 #pragma unroll
     for (int k = 0; k < BATCH; k++) {
-      const int i = i0 + k * 256;
+      const int i = i0 + k * nt;
       if (i >= nA) continue;
 #pragma unroll
       for (int g = 0; g < G; g++) {
@@ -1181,38 +1186,41 @@ __device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
   __syncthreads();
 }
 
-// out = (A_0 + w A_1) / (L_0 + w L_1) for unit u from its records, with part 1
-// weighted by w = N_tail / b when the tail was sampled (1 otherwise). One
-// thread per (head, dimension) folds the records of each part in order with
-// a running maximum (the record loads do not depend on the fold, so they run
-// ahead of it).
+// out = (A_0 + w A_1) / (L_0 + w L_1) for unit u, head g from its records,
+// with part 1 weighted by w = N_tail / b when the tail was sampled (1
+// otherwise). Block of kCombGroups * D threads: thread (r, e) folds every
+// kCombGroups-th record of each list with a running maximum (batches of
+// loads issued ahead of the fold), and the groups' states are then merged.
+constexpr int kCombGroups = 4;
+
 template <int D, int G, int MODE>
-__device__ void unit_combine(const DevParams& P, int u) {
+__device__ void unit_combine(const DevParams& P, int u, int g) {
   constexpr int REC = G * (2 + D);
+  __shared__ float s_st[2][kCombGroups][3][D];
   const UnitInfo inf = P.info[u];
   const int b = u / P.Hkv, h = u % P.Hkv;
-  const int g = threadIdx.x / D, e = threadIdx.x % D;
+  const int r = threadIdx.x / D, e = threadIdx.x % D;
   const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
   const bool sampled = MODE == kModeSample && inf.mode == 2 && !inf.exhausted;
-  float M[2], L[2], A[2];
 #pragma unroll
   for (int part = 0; part < 2; part++) {
     float m = -INFINITY, l = 0.0f, a = 0.0f;
     auto fold = [&](const long long* pre, const float* rec, int C) {
       int cf, cl;
       slice_ctas(pre, 2 * u + part, pre[2 * P.units], C, cf, cl);
-      constexpr int B = 8;  // records loaded together, then folded
-      for (int c0 = cf; c0 <= cl; c0 += B) {
+      constexpr int B = 4;  // records loaded together, then folded
+      for (int c0 = cf + r; c0 <= cl; c0 += B * kCombGroups) {
         float rm[B], rl[B], ra[B];
 #pragma unroll
         for (int j = 0; j < B; j++) {
+          const int c = c0 + j * kCombGroups;
           rm[j] = -INFINITY;
           rl[j] = ra[j] = 0.0f;
-          if (c0 + j <= cl) {
-            const float* r = rec + static_cast<size_t>(c0 + j + 2 * u + part) * REC + g * (2 + D);
-            rm[j] = r[0];
-            rl[j] = r[1];
-            ra[j] = r[2 + e];
+          if (c <= cl) {
+            const float* q = rec + static_cast<size_t>(c + 2 * u + part) * REC + g * (2 + D);
+            rm[j] = q[0];
+            rl[j] = q[1];
+            ra[j] = q[2 + e];
           }
         }
 #pragma unroll
@@ -1232,6 +1240,25 @@ __device__ void unit_combine(const DevParams& P, int u) {
       if (!(part == 1 && whole_tail)) fold(P.pre_det, P.rec_det, P.CD);
     } else {
       fold(P.pre_det, P.rec_det, P.CD);
+    }
+    s_st[part][r][0][e] = m;
+    s_st[part][r][1][e] = l;
+    s_st[part][r][2][e] = a;
+  }
+  __syncthreads();
+  if (r != 0) return;
+  float M[2], L[2], A[2];
+#pragma unroll
+  for (int part = 0; part < 2; part++) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kCombGroups; q++) m = fmaxf(m, s_st[part][q][0][e]);
+    float l = 0.0f, a = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kCombGroups; q++) {
+      const float sc = exp_rel(s_st[part][q][0][e], m);
+      l += s_st[part][q][1][e] * sc;
+      a += s_st[part][q][2][e] * sc;
     }
     M[part] = m;
     L[part] = l;
@@ -1630,9 +1657,36 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
   }
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
   const unsigned bb = static_cast<unsigned>(u / P.Hkv), hh = static_cast<unsigned>(u % P.Hkv);
-  for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
-    const int rho = whole_tail ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
-    sel[t] = tail_position(topk, inf.k, inf.s1, rho);
+  const int step0 = inf.k > 0 ? 1 << (31 - __clz(inf.k)) : 0;
+  // each thread takes aligned groups of four draws: one Philox block serves
+  // all four, and their four searches advance together
+  for (int t4 = (t0 & ~3) + 4 * static_cast<int>(threadIdx.x); t4 < t1; t4 += 4 * static_cast<int>(blockDim.x)) {
+    int rho[4];
+    if (whole_tail) {
+#pragma unroll
+      for (int j = 0; j < 4; j++) rho[j] = t4 + j;
+    } else {
+      const uint4 q = draw_block(P.seed, bb, hh, static_cast<unsigned>(t4) >> 2);
+      rho[0] = lemire(q.x, inf.ntail);
+      rho[1] = lemire(q.y, inf.ntail);
+      rho[2] = lemire(q.z, inf.ntail);
+      rho[3] = lemire(q.w, inf.ntail);
+    }
+    // c_j = #{i : topk[i] - s1 - i <= rho_j} by binary lifting (the left side
+    // is non-decreasing in i)
+    int c[4] = {0, 0, 0, 0};
+    for (int step = step0; step > 0; step >>= 1) {
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int i = c[j] + step;
+        if (i <= inf.k && topk[i - 1] - inf.s1 - (i - 1) <= rho[j]) c[j] = i;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int t = t4 + j;
+      if (t >= t0 && t < t1) sel[t] = inf.s1 + rho[j] + c[j];
+    }
   }
   __syncthreads();
 }
@@ -1648,7 +1702,7 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
 //   ascending (ties at the threshold to the lowest positions, as the key's
 //   low half orders them). The sorted list, kept in shared memory, then
 //   serves the pilot draws (or the whole tail when it is no larger than the
-//   pilot), as in k_draws<0>.
+//   pilot), as k_draws does after the other selections.
 constexpr int kSel1Threads = 1024;
 constexpr int kSel1MaxKeys = 45056;
 constexpr int kSel1Cand = kTopkSmem - kHist2;  // candidate slots; with the histogram, the top-k staging
@@ -1810,68 +1864,66 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
 }
 
 // ============================================================ k_draws
-// Positions of sampled entries, one thread per entry. PHASE 0 (before the det
-// gather): the p pilot draws, or the whole tail when it is no larger than the
-// pilot. PHASE 1 (after the budget): draws t in [p, b), or the whole tail
-// when the budget covers it. Grid (units, splits).
-template <int PHASE>
+// Positions of the pilot draws (or of the whole tail when it is no larger
+// than the pilot), one thread per entry, after the cluster or grid-wide top-k
+// selection (k_select1 does this itself). Grid (units, splits).
 __global__ void __launch_bounds__(256) k_draws(DevParams P) {
   __shared__ int s_topk[kTopkSmem];
   grid_dependency_wait();
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
-  int t0 = 0, t1 = 0;
-  bool whole = false;
-  if (PHASE == 0) {
-    if (inf.mode == 2) t1 = inf.p;
-    if (inf.mode == 1) {
-      t1 = inf.ntail;
-      whole = true;
-    }
-  } else if (inf.mode == 2) {
-    if (inf.exhausted) {
-      t1 = inf.ntail;
-      whole = true;
-    } else {
-      t0 = inf.p;
-      t1 = inf.bsz;
-    }
-  }
-  if (PHASE == 1 && blockIdx.x == 0 && blockIdx.y == 0) {
-    // slice prefix of the sample gather (every unit's budget is known now)
-    __shared__ unsigned s_warp[32];
-    __shared__ long long s_carry;
-    write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
-    __syncthreads();
-  }
-  const int n = t1 - t0;
-  const int a = t0 + static_cast<int>(static_cast<long long>(n) * blockIdx.y / gridDim.y);
-  const int e = t0 + static_cast<int>(static_cast<long long>(n) * (blockIdx.y + 1) / gridDim.y);
-  if (a < e) write_draw_positions(P, u, inf, whole, a, e, s_topk);
+  const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
+  const int a = static_cast<int>(static_cast<long long>(t1) * blockIdx.y / gridDim.y);
+  const int e = static_cast<int>(static_cast<long long>(t1) * (blockIdx.y + 1) / gridDim.y);
+  if (a < e) write_draw_positions(P, u, inf, inf.mode == 1, a, e, s_topk);
   grid_dependents_launch();
 }
 
 // ============================================================ k_budget
 // One CTA per unit: the per-head CLT budget from the det gather's records
 // (score maxima) and true scores.
+// The same CTA then writes the positions of the rest of the sample (draws t
+// in [p, b), or the whole tail when the budget covers it), and the grid's
+// last CTA to finish writes the sample gather's slice prefix (the arrival
+// counter is zeroed by k_prep).
+constexpr int kBudgetThreads = 512;
 template <int D, int G>
-__global__ void __launch_bounds__(256) k_budget(DevParams P) {
+__global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
   __shared__ float s_mh[G];
+  __shared__ int s_topk[kTopkSmem];
+  __shared__ unsigned s_warp[32];
+  __shared__ long long s_carry;
+  __shared__ bool s_last;
   grid_dependency_wait();
   const int u = blockIdx.x;
-  const UnitInfo inf = P.info[u];
+  UnitInfo inf = P.info[u];
   if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
   unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
+  if (inf.mode == 2) {
+    inf = P.info[u];  // with the budget (written by this CTA)
+    if (inf.exhausted) write_draw_positions(P, u, inf, true, 0, inf.ntail, s_topk);
+    else if (inf.bsz > inf.p) write_draw_positions(P, u, inf, false, inf.p, inf.bsz, s_topk);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this unit's state before the arrival
+    s_last = atomicAdd(P.gcnt, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
+  }
   grid_dependents_launch();
 }
 
 // ============================================================ k_combine
-// One CTA per unit, one thread per (head, dimension): merge the unit's
-// records and write the output.
+// One CTA per (unit, head), kCombGroups threads per dimension: merge the
+// unit's records and write the output.
 template <int D, int G, int MODE>
-__global__ void __launch_bounds__(G * D) k_combine(DevParams P) {
+__global__ void __launch_bounds__(kCombGroups * D) k_combine(DevParams P) {
   grid_dependency_wait();
-  unit_combine<D, G, MODE>(P, blockIdx.x);
+  unit_combine<D, G, MODE>(P, blockIdx.x, blockIdx.y);
   grid_dependents_launch();
 }
 
