@@ -24,7 +24,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from verified_sparse_attention_b200 import _abi, synth  # noqa: E402
+from verified_sparse_attention_b200 import _abi, ranks, synth  # noqa: E402
 from verified_sparse_attention_b200.decoder import decoder_for, params_for  # noqa: E402
 
 METRIC = "sparse decode-attn calls/s & achieved HBM GB/s (% of ~8 TB/s) at 32k–128k ctx"
@@ -140,8 +140,7 @@ def run_gpu_arm(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[args.workload]
-    if rank:
-        w = w.replace(data_seed=w.data_seed + 1000 * rank)
+    w = ranks.rank_workload(w, rank)
     x = synth.make_inputs(w, device=dev)
     dec = decoder_for(w, device=dev)
     prm = params_for(w, x, eps=args.eps)
@@ -168,8 +167,7 @@ def run_gpu_arm(args, rank, world, local_rank):
     _abi.vattn_score_pass_ms(dec.ctx, reset=True)
     _abi.vattn_set_timing(dec.ctx, True)
 
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
@@ -178,16 +176,11 @@ def run_gpu_arm(args, rank, world, local_rank):
             step()
         t1.record(stream)
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier(world)
     _abi.vattn_set_timing(dec.ctx, False)
     ms = t0.elapsed_time(t1)
     score_ms, score_n = _abi.vattn_score_pass_ms(dec.ctx, reset=True)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = ranks.max_over_ranks(ms, world, dev)
 
     score_bytes, call_bytes = algorithmic_bytes(w, x, outs)
     budgets = outs["budgets"].cpu()
@@ -240,21 +233,16 @@ def run_e2e(args, w, x, dec, prm, stream, dev, world):
 
     step()
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    ranks.barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(steps):
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = ranks.max_over_ranks(a.elapsed_time(b), world, dev)
     del devb, host
-    return {"value": world * steps / (ms / 1e3), "unit": "calls/s",
+    return {"value": ranks.job_rate(world, steps, ms), "unit": "calls/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
@@ -298,9 +286,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = ranks.rank_env()
     w = synth.WORKLOADS[args.workload]
     if args.eps is not None:
         w = w.replace(eps=args.eps)
@@ -309,7 +295,7 @@ def main():
            "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
 
     if args.impl == "reference":
-        if rank != 0:
+        if not ranks.reports(rank):
             return
         t_gen = time.perf_counter()
         cpu = synth.make_inputs(w)
@@ -340,7 +326,7 @@ def main():
     dec, r = run_gpu_arm(args, rank, world, local_rank)
     peak, peak_kind = load_peaks()
     w = r["w"]
-    calls_s = world * args.steps / (r["ms"] / 1e3)
+    calls_s = ranks.job_rate(world, args.steps, r["ms"])
     avg_score_s = (r["score_ms"] / max(1, r["score_n"])) / 1e3
     achieved = r["score_bytes"] / avg_score_s / 1e9
     call_s = r["ms"] / 1e3 / args.steps
@@ -367,10 +353,10 @@ def main():
                                 "sample": f"{done} (sequence, KV head) units of a {w.units}-unit call "
                                           f"in {el:.1f}s, single-threaded C oracle"}
     dec.close()
-    if rank == 0:
+    if ranks.reports(rank):
         emit(line)
     if world > 1:
-        torch.distributed.barrier()
+        ranks.barrier(world)
         torch.distributed.destroy_process_group()
 
 
