@@ -522,10 +522,11 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
       launch(vattn::k_sel_count, seg_grid, dim3(256), 0, st, P, &launches);
       launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
     }
-    launch(vattn::k_draws, dim3(P.units, ctx->draw_splits), dim3(256), 0, st, P, &launches);
+    launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(128), 0, st, P, &launches);
   }
   launch(K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(vattn::kBudgetThreads), 0, st, P, &launches);
+  launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(128), 0, st, P, &launches);
   launch(K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   launch(K.combine_sample, dim3(P.units, ctx->G), dim3(vattn::kCombGroups * c.head_dim), 0, st, P, &launches);
   return finish(ctx, launches);

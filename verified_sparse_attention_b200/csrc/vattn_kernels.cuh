@@ -1864,46 +1864,49 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
 }
 
 // ============================================================ k_draws
-// Positions of the pilot draws (or of the whole tail when it is no larger
-// than the pilot), one thread per entry, after the cluster or grid-wide top-k
-// selection (k_select1 does this itself). Grid (units, splits).
-__global__ void __launch_bounds__(256) k_draws(DevParams P) {
+// Positions of sampled entries. PHASE 0: the pilot draws (or the whole tail
+// when it is no larger than the pilot), after the cluster or grid-wide top-k
+// selection (k_select1 does this itself). PHASE 1, after the budget: draws t
+// in [p, b), or the whole tail when the budget covers it. Grid (units, splits).
+template <int PHASE>
+__global__ void __launch_bounds__(128) k_draws(DevParams P) {
   __shared__ int s_topk[kTopkSmem];
   grid_dependency_wait();
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
-  const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
-  const int a = static_cast<int>(static_cast<long long>(t1) * blockIdx.y / gridDim.y);
-  const int e = static_cast<int>(static_cast<long long>(t1) * (blockIdx.y + 1) / gridDim.y);
-  if (a < e) write_draw_positions(P, u, inf, inf.mode == 1, a, e, s_topk);
+  int t0 = 0, t1 = 0;
+  bool whole = false;
+  if (PHASE == 0) {
+    t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
+    whole = inf.mode == 1;
+  } else if (inf.mode == 2) {
+    whole = inf.exhausted != 0;
+    t0 = whole ? 0 : inf.p;
+    t1 = whole ? inf.ntail : inf.bsz;
+  }
+  const int a = t0 + static_cast<int>(static_cast<long long>(t1 - t0) * blockIdx.y / gridDim.y);
+  const int e = t0 + static_cast<int>(static_cast<long long>(t1 - t0) * (blockIdx.y + 1) / gridDim.y);
+  if (a < e) write_draw_positions(P, u, inf, whole, a, e, s_topk);
   grid_dependents_launch();
 }
 
 // ============================================================ k_budget
 // One CTA per unit: the per-head CLT budget from the det gather's records
 // (score maxima) and true scores.
-// The same CTA then writes the positions of the rest of the sample (draws t
-// in [p, b), or the whole tail when the budget covers it), and the grid's
-// last CTA to finish writes the sample gather's slice prefix (the arrival
-// counter is zeroed by k_prep).
+// The grid's last CTA to finish writes the sample gather's slice prefix (the
+// arrival counter is zeroed by k_prep).
 constexpr int kBudgetThreads = 512;
 template <int D, int G>
 __global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
   __shared__ float s_mh[G];
-  __shared__ int s_topk[kTopkSmem];
   __shared__ unsigned s_warp[32];
   __shared__ long long s_carry;
   __shared__ bool s_last;
   grid_dependency_wait();
   const int u = blockIdx.x;
-  UnitInfo inf = P.info[u];
+  const UnitInfo inf = P.info[u];
   if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
   unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
-  if (inf.mode == 2) {
-    inf = P.info[u];  // with the budget (written by this CTA)
-    if (inf.exhausted) write_draw_positions(P, u, inf, true, 0, inf.ntail, s_topk);
-    else if (inf.bsz > inf.p) write_draw_positions(P, u, inf, false, inf.p, inf.bsz, s_topk);
-  }
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();  // this unit's state before the arrival
