@@ -334,7 +334,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic", "config": cfg,
-            "roofline": {"bound": "hbm", "kernel": "score pass (k_score_rows / k_score_sparq)",
+            "roofline": {"bound": "hbm", "kernel": "score pass (k_score_tma / k_score_rows / k_score_sparq)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": achieved / peak,
                          "traffic": profiled_traffic(w.name),

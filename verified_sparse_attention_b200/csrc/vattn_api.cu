@@ -22,6 +22,8 @@ struct vattn_ctx {
   int units_max = 0;
   int nseg = 0;
   int score_grid = 0;
+  bool score_tma = false;   // contiguous cache: the bulk-copy score pass
+  size_t score_smem = 0;
   int gather_grid = 0;     // CTAs of each gather launch
   int CD = 0, CS = 0;      // record producers (warps) of the det/dense and sample gathers
   size_t gather_smem = 0;   // gathers (all modes)
@@ -126,6 +128,9 @@ struct Kernels {
   void (*score_exact)(DevParams);
   void (*score_loki)(DevParams);
   void (*score_sparq)(DevParams);
+  void (*score_exact_tma)(DevParams);  // contiguous caches
+  void (*score_loki_tma)(DevParams);
+  size_t score_tma_smem, score_loki_tma_smem;
   void (*det)(DevParams);
   void (*sample)(DevParams);
   void (*dense)(DevParams);
@@ -142,6 +147,10 @@ Kernels kernels_for() {
   k.prep = vattn::k_prep<T, D, G>;
   k.score_exact = vattn::k_score_rows<T, D>;
   k.score_loki = vattn::k_score_rows<T, 32>;
+  k.score_exact_tma = vattn::k_score_tma<T, D>;
+  k.score_loki_tma = vattn::k_score_tma<T, 32>;
+  k.score_tma_smem = vattn::ScoreShape<T, D>::SMEM;
+  k.score_loki_tma_smem = vattn::ScoreShape<T, 32>::SMEM;
   k.score_sparq = vattn::k_score_sparq<T, D>;
   k.det = vattn::k_gather<T, D, G, vattn::kModeDet>;
   k.sample = vattn::k_gather<T, D, G, vattn::kModeSample>;
@@ -220,6 +229,8 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->hist = ctx->hist;
   P->segcnt = ctx->segcnt;
   P->pscore = ctx->pscore;
+  // only the grid-wide select reads the digit-2 and digit-3 histograms
+  P->hist_words = (ctx->select1 || ctx->select_smem) ? vattn::kHist1 : vattn::kHistAll;
   P->prefix = ctx->prefix;
   P->cnt = ctx->cnt;
   P->gcnt = ctx->gcnt;
@@ -301,6 +312,16 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
   ctx->score_grid = (occ < 1 ? 1 : occ) * ctx->num_sms;
+  if (cfg->page_size >= cfg->max_ctx && cfg->proxy != VATTN_SPARQ) {
+    void (*tma)(DevParams) = cfg->proxy == VATTN_LOKI ? K.score_loki_tma : K.score_exact_tma;
+    const size_t smem = cfg->proxy == VATTN_LOKI ? K.score_loki_tma_smem : K.score_tma_smem;
+    if (cudaFuncSetAttribute(tma, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+        cudaSuccess) {
+      ctx->score_tma = true;
+      ctx->score_smem = smem;
+    }
+    cudaGetLastError();
+  }
   ctx->gather_smem = K.gather_smem;
   ctx->gather_threads = K.gather_threads;
   for (auto fn : {K.det, K.sample, K.dense})
@@ -506,7 +527,11 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     }
     cudaEventRecord(ctx->ev_start[ctx->ev_used], st);
   }
-  launch(score, dim3(ctx->score_grid), dim3(256), 0, st, P, &launches);
+  if (ctx->score_tma)
+    launch(c.proxy == VATTN_LOKI ? K.score_loki_tma : K.score_exact_tma, dim3(ctx->num_sms), dim3(256),
+           ctx->score_smem, st, P, &launches);
+  else
+    launch(score, dim3(ctx->score_grid), dim3(256), 0, st, P, &launches);
   if (timed) {
     cudaEventRecord(ctx->ev_stop[ctx->ev_used], st);
     ctx->ev_used++;

@@ -87,6 +87,7 @@ struct DevParams {
   unsigned* hist;   // [units][kHistAll]
   unsigned* segcnt; // [units][nseg][2]
   float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
+  int hist_words;   // histogram words per unit that k_prep zeroes (all only for the grid-wide select)
   long long* prefix;// [units + 1]: score-pass work prefix
   unsigned* cnt;    // [units][2]: finished-segment counters of the det and sample gathers
   unsigned* gcnt;   // finished-CTA counter of the det gather

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   }
 
   unsigned* hist = P.hist + static_cast<size_t>(u) * kHistAll;
-  for (int i = tid; i < kHistAll; i += blockDim.x) hist[i] = 0u;
+  for (int i = tid; i < P.hist_words; i += blockDim.x) hist[i] = 0u;
   if (tid < 2) P.cnt[2 * u + tid] = 0u;
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
   for (int i = tid; i < r.s1; i += blockDim.x) sel[i] = i;
@@ -247,14 +247,15 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
 }
 
 // ============================================================ score pass helpers
-// Find the unit whose work range contains item `x` (prefix is non-decreasing).
-__device__ __forceinline__ int find_unit(const long long* prefix, int units, long long x) {
-  int lo = 0, hi = units;  // largest u with prefix[u] <= x
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= x) lo = mid; else hi = mid;
-  }
-  return lo;
+// The whole block searches the prefix in one round of loads: the unit
+// whose non-empty range [prefix[u], prefix[u+1]) holds x (0 if none).
+__device__ __forceinline__ int find_unit_block(const long long* prefix, int units, long long x, int* s_u) {
+  if (threadIdx.x == 0) *s_u = 0;
+  __syncthreads();
+  for (int v = threadIdx.x; v < units; v += blockDim.x)
+    if (prefix[v] <= x && x < prefix[v + 1]) *s_u = v;
+  __syncthreads();
+  return *s_u;
 }
 
 __device__ __forceinline__ void flush_hist(unsigned* s_hist, unsigned* g_hist) {
@@ -296,7 +297,8 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
   const long long beg = total * blockIdx.x / gridDim.x;
   const long long end = total * (blockIdx.x + 1) / gridDim.x;
   if (beg >= end) return;
-  int u = find_unit(P.prefix, P.units, beg);
+  __shared__ int s_u;
+  int u = find_unit_block(P.prefix, P.units, beg, &s_u);
   long long cur = beg;
   while (cur < end) {
     while (P.prefix[u + 1] <= cur) u++;
@@ -358,7 +360,8 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
   const long long end = total * (blockIdx.x + 1) / gridDim.x;
   if (beg >= end) return;
   const int r = P.rank;
-  int u = find_unit(P.prefix, P.units, beg);
+  __shared__ int s_u;
+  int u = find_unit_block(P.prefix, P.units, beg, &s_u);
   long long cur = beg;
   while (cur < end) {
     while (P.prefix[u + 1] <= cur) u++;
@@ -1276,6 +1279,134 @@ __device__ void unit_combine(const DevParams& P, int u, int g) {
   *out = (A[0] * c0 + w * (A[1] * c1)) / (L[0] * c0 + w * (L[1] * c1));
 }
 
+
+// ============================================================ k_score_tma
+// The exact / Loki score pass for a contiguous cache (one page per sequence,
+// so a unit's middle rows are consecutive in memory): every warp streams
+// blocks of BLK consecutive rows (8 KB) through a private ring of NS shared-
+// memory stages, one bulk copy per block issued NS - 1 blocks ahead, and
+// computes each row's dot from shared memory exactly as k_score_rows does
+// (the same chunk chains and the same transposed reduction).
+template <typename T, int W>
+struct ScoreShape {
+  static constexpr int E = Elem<T>::kPer16;
+  static constexpr int L = W / E;                  // lanes (16-byte chunks) per row
+  static constexpr int RPW = 32 / L;               // rows per warp-wide load
+  static constexpr int U = L < 8 ? L : 8;          // rows per lane group per step
+  static constexpr int ROWS_STEP = RPW * U;
+  static constexpr int ROWB = W * static_cast<int>(sizeof(T));
+  static constexpr int BLKB = 8192;
+  static constexpr int BLK = BLKB / ROWB;          // rows per block
+  static constexpr int STEPS = BLK / ROWS_STEP;
+  static constexpr int NW = 8, NS = 3;
+  static constexpr size_t OFF_BAR = static_cast<size_t>(NW) * NS * BLKB;  // 192 KB of rings
+  static constexpr size_t SMEM = OFF_BAR + static_cast<size_t>(NW) * NS * 8;
+  static_assert(BLK % ROWS_STEP == 0, "whole steps per block");
+};
+
+template <typename T, int W>
+__global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevParams P) {
+  using S = ScoreShape<T, W>;
+  constexpr int E = S::E, L = S::L, RPW = S::RPW, U = S::U, ROWB = S::ROWB, BLK = S::BLK, NS = S::NS,
+                NW = S::NW;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ unsigned s_hist[kHist1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / L, li = lane % L;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR) + warp * NS;
+  unsigned char* ring = smem + static_cast<size_t>(warp) * NS * S::BLKB;
+  if (lane < NS) mbar_init(&bars[lane], 1);
+  for (int i = threadIdx.x; i < kHist1; i += blockDim.x) s_hist[i] = 0u;
+  mbar_init_fence();
+  __syncthreads();
+  grid_dependency_wait();
+  const bool loki = P.proxy == kProxyLoki;
+  const T* cache = static_cast<const T*>(loki ? P.kp : P.k);
+  const float* qsrc = loki ? P.qsel : P.qbar;
+
+  const long long total = P.prefix[P.units];
+  const long long beg = total * blockIdx.x / gridDim.x;
+  const long long end = total * (blockIdx.x + 1) / gridDim.x;
+  if (beg >= end) return;
+  __shared__ int s_u;
+  int u = find_unit_block(P.prefix, P.units, beg, &s_u);
+  long long cur = beg;
+  unsigned issued = 0;  // blocks this warp issued so far (stage and phase follow from it)
+  bool failed = false;
+  while (cur < end) {
+    while (P.prefix[u + 1] <= cur) u++;
+    const long long uend = min(end, P.prefix[u + 1]);
+    const UnitInfo inf = P.info[u];
+    if (inf.n > 0) {
+      const int b = u / P.Hkv, h = u % P.Hkv;
+      const int j0 = inf.s1 + static_cast<int>(cur - P.prefix[u]);
+      const int nrow = static_cast<int>(uend - cur);
+      float q[E];
+#pragma unroll
+      for (int e = 0; e < E; e++) q[e] = qsrc[static_cast<size_t>(u) * P.D + li * E + e];
+      // the sequence's one page: row j of the unit at rows + j * W
+      const size_t page = static_cast<size_t>(P.page_table[static_cast<size_t>(b) * P.pps]);
+      const T* rows = cache + (page * P.Hkv + h) * P.ps * static_cast<size_t>(W);
+      unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
+      const int nblk = (nrow + BLK - 1) / BLK;
+      const int nbw = (!failed && warp < nblk) ? (nblk - warp + NW - 1) / NW : 0;  // blocks warp + t * NW
+      int nis = 0;
+      auto issue = [&](int t) {
+        const int r0 = (warp + t * NW) * BLK;
+        const int n = min(BLK, nrow - r0);
+        const unsigned g = issued + static_cast<unsigned>(t);
+        const int st = static_cast<int>(g % NS);
+        fence_proxy_async();  // this lane's reads of the stage come before the copy's writes
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(n * ROWB));
+          bulk_copy_g2s(ring + st * S::BLKB, rows + static_cast<size_t>(j0 + r0) * W,
+                        static_cast<unsigned>(n * ROWB), &bars[st]);
+        }
+        nis++;
+      };
+#pragma unroll 1
+      for (int t = 0; t < NS - 1 && t < nbw; t++) issue(t);
+#pragma unroll 1
+      for (int t = 0; t < nbw; t++) {
+        if (t + NS - 1 < nbw && !failed) issue(t + NS - 1);
+        if (t >= nis) continue;  // never issued (only after a failed wait)
+        const unsigned g = issued + static_cast<unsigned>(t);
+        const int st = static_cast<int>(g % NS);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
+          if (!failed && lane == 0) atomicOr(P.err, kDevTimeout);
+          failed = true;
+        }
+        if (failed) continue;
+        const unsigned char* sb = ring + st * S::BLKB;
+        const int r0 = (warp + t * NW) * BLK;
+        const int n = min(BLK, nrow - r0);
+#pragma unroll
+        for (int step = 0; step < S::STEPS; step++) {
+          float a[U];
+#pragma unroll
+          for (int k = 0; k < U; k++) {
+            const int r = step * S::ROWS_STEP + k * RPW + grp;
+            const uint4 raw = r < n ? *reinterpret_cast<const uint4*>(sb + r * ROWB + li * 16)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            a[k] = chunk_dot<T>(q, raw);
+          }
+          const float sc = reduce_rows<L, U>(a, li);
+          const int r = step * S::ROWS_STEP + reduce_rows_row<L, U>(li) * RPW + grp;
+          if ((li % (L / U)) == 0 && r < n) {
+            const unsigned o = ord_key(sc);
+            ordk[j0 + r0 + r] = o;
+            atomicAdd(&s_hist[o >> 21], 1u);
+          }
+        }
+        __syncwarp();  // the stage is free again
+      }
+      issued += static_cast<unsigned>(nbw);
+      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
+    }
+    cur = uend;
+  }
+}
 
 // ============================================================ k_gather
 template <typename T, int D, int G, int MODE>
