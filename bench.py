@@ -246,6 +246,31 @@ def run_e2e(args, w, x, dec, prm, stream, dev, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
+def time_oracle_all_cores(w, cpu_inputs, budget_s):
+    """The same oracle on every host core: one thread per core, each running whole
+    (sequence, KV head) units (the C library releases the GIL) until budget_s.
+    Returns (calls/s equivalent, units done, seconds, threads)."""
+    import concurrent.futures
+    import oracle
+    pr = oracle.make_problem(w)
+    U = w.units
+    T = os.cpu_count() or 1
+    t0 = time.perf_counter()
+
+    def worker(tid):
+        done, u = 0, tid
+        while time.perf_counter() - t0 < budget_s and done < 5 * U:
+            oracle.decode(pr, cpu_inputs, units=[u % U])
+            done += 1
+            u += T
+        return done
+
+    with concurrent.futures.ThreadPoolExecutor(T) as ex:
+        done = sum(ex.map(worker, range(T)))
+    el = time.perf_counter() - t0
+    return (done / U) / el, done, el, T
+
+
 def time_oracle(w, cpu_inputs, budget_s, units_per_step=None):
     """Run the oracle unit by unit on the host until budget_s elapses (or all units).
     Returns (calls/s equivalent, units done, seconds)."""
@@ -352,6 +377,10 @@ def main():
         line["cpu_baseline"] = {"value": val, "unit": "calls/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} (sequence, KV head) units of a {w.units}-unit call "
                                           f"in {el:.1f}s, single-threaded C oracle"}
+        val, done, el, T = time_oracle_all_cores(w, cpu, args.cpu_budget_s)
+        line["cpu_baseline_all_cores"] = {
+            "value": val, "unit": "calls/s", "cores": T, "kind": "oracle",
+            "sample": f"{done} units in {el:.1f}s, one unit per call on {T} threads of the same C oracle"}
     dec.close()
     if ranks.reports(rank):
         emit(line)
