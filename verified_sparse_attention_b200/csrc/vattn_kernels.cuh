@@ -390,13 +390,14 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
 #pragma unroll
         for (int v = 0; v < V; v++) acc[v] = 0.0f;
         int t = 0;
-        for (; t + 8 <= r; t += 8) {
-          uint4 raw[8];
+        constexpr int NB = 16;  // dims loaded together (16-byte vectors in flight per thread)
+        for (; t + NB <= r; t += NB) {
+          uint4 raw[NB];
 #pragma unroll
-          for (int c = 0; c < 8; c++)
+          for (int c = 0; c < NB; c++)
             raw[c] = ld_stream(kt + rowbase + static_cast<size_t>(s_dim[t + c]) * ps + off);
 #pragma unroll
-          for (int c = 0; c < 8; c++) {
+          for (int c = 0; c < NB; c++) {
             float x[V];
             Elem<T>::unpack(raw[c], x);
             const float qv = s_qv[t + c];
