@@ -1880,22 +1880,32 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
       s_krem = inf.k;
       s_ncand = 0;
     }
-    if (nbody > 0 && !__all_sync(0xffffffffu, mbar_wait(&s_bar, 0u)) && lane == 0)
-      atomicOr(P.err, kDevTimeout);
     __syncthreads();
+    // digit 1 while the keys are still arriving
     find_digit_bt<kHist1, kSel1Threads>(s_hist, inf.k, &s_digit, &s_krem, s_warp);
     const unsigned d1 = static_cast<unsigned>(s_digit);
     const int krem1 = s_krem;
+    if (nbody > 0 && !__all_sync(0xffffffffu, mbar_wait(&s_bar, 0u)) && lane == 0)
+      atomicOr(P.err, kDevTimeout);
 
     // digit 2 over the keys of bin d1, collecting them
     for (int x = tid; x < kHist2; x += kSel1Threads) s_hist[x] = 0u;
-    __syncthreads();
-    for (int x = tid; x < mlen; x += kSel1Threads) {
-      const unsigned o = s_keys[x];
-      if ((o >> 21) == d1) {
-        atomicAdd(&s_hist[(o >> 10) & 2047u], 1u);
-        const unsigned slot = atomicAdd(&s_ncand, 1u);
-        if (slot < static_cast<unsigned>(kSel1Cand)) s_cand[slot] = static_cast<unsigned>(x);
+    __syncthreads();  // also: every thread's copy wait is over, the keys are visible
+    for (int x0 = tid; x0 < mlen; x0 += 8 * kSel1Threads) {
+      unsigned o[8];
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const int x = x0 + i * kSel1Threads;
+        o[i] = x < mlen ? s_keys[x] : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const int x = x0 + i * kSel1Threads;
+        if (x < mlen && (o[i] >> 21) == d1) {
+          atomicAdd(&s_hist[(o[i] >> 10) & 2047u], 1u);
+          const unsigned slot = atomicAdd(&s_ncand, 1u);
+          if (slot < static_cast<unsigned>(kSel1Cand)) s_cand[slot] = static_cast<unsigned>(x);
+        }
       }
     }
     __syncthreads();
