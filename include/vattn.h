@@ -163,12 +163,14 @@ int vattn_last_error(vattn_ctx* ctx, int sync);
 /* Bytes of device workspace the context holds. */
 size_t vattn_workspace_bytes(const vattn_ctx* ctx);
 
-/* Per-call kernel timing: when enabled, vattn_decode records a CUDA event
-   pair around its dominant kernel (the ranking-score pass) on `stream`;
-   vattn_score_pass_ms returns the summed elapsed time in milliseconds since
-   the last reset and how many passes it covers. Calls synchronise on the
-   recorded events (host wait). */
-int vattn_set_timing(vattn_ctx* ctx, int enable);
+/* Per-call kernel timing: with period >= 1, every period-th vattn_decode call
+   records a CUDA event pair around its dominant kernel (the ranking-score
+   pass) on `stream` (0 turns it off; the event pair breaks the overlap of
+   that kernel with its neighbours, so sampling keeps the other calls
+   undisturbed); vattn_score_pass_ms returns the summed elapsed time in
+   milliseconds since the last reset and how many passes it covers. Calls
+   synchronise on the recorded events (host wait). */
+int vattn_set_timing(vattn_ctx* ctx, int period);
 int vattn_score_pass_ms(vattn_ctx* ctx, double* total_ms, int* count, int reset);
 
 /* Number of kernel launches the last vattn_decode / vattn_dense_decode call

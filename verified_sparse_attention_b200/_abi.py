@@ -149,8 +149,9 @@ def vattn_workspace_bytes(ctx):
     return lib().vattn_workspace_bytes(ctx)
 
 
-def vattn_set_timing(ctx, enable):
-    return _check(lib().vattn_set_timing(ctx, 1 if enable else 0), "vattn_set_timing")
+def vattn_set_timing(ctx, period):
+    """Time the score pass of every `period`-th decode call (True = every call, 0 / False = off)."""
+    return _check(lib().vattn_set_timing(ctx, int(period)), "vattn_set_timing")
 
 
 def vattn_score_pass_ms(ctx, reset=True):

@@ -56,7 +56,8 @@ struct vattn_ctx {
   double cached_delta = -1.0;
   double cached_z = 0.0;
   // timing of the score pass
-  int timing = 0;
+  int timing = 0;            // period (0: off)
+  long long timing_calls = 0;
   std::vector<cudaEvent_t> ev_start, ev_stop;
   size_t ev_used = 0;
 };
@@ -414,9 +415,10 @@ size_t vattn_workspace_bytes(const vattn_ctx* ctx) { return ctx ? ctx->ws_bytes 
 
 int vattn_last_launch_count(const vattn_ctx* ctx) { return ctx ? ctx->last_launches : 0; }
 
-int vattn_set_timing(vattn_ctx* ctx, int enable) {
-  if (!ctx) return VATTN_EINVAL;
-  ctx->timing = enable ? 1 : 0;
+int vattn_set_timing(vattn_ctx* ctx, int period) {
+  if (!ctx || period < 0) return VATTN_EINVAL;
+  ctx->timing = period;
+  ctx->timing_calls = 0;
   return VATTN_OK;
 }
 
@@ -516,7 +518,7 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
   void (*score)(DevParams) = c.proxy == VATTN_SPARQ ? K.score_sparq
                              : c.proxy == VATTN_LOKI ? K.score_loki : K.score_exact;
-  const bool timed = ctx->timing != 0;
+  const bool timed = ctx->timing > 0 && (ctx->timing_calls++ % ctx->timing) == 0;
   if (timed) {
     if (ctx->ev_used == ctx->ev_start.size()) {
       cudaEvent_t a, b;
