@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
     if (tid == 0) {
       P.pre_det[ns] = carry;
       P.gcnt[0] = 0u;
+      P.gcnt[1] = 0u;
     }
     return;
   }
@@ -247,6 +248,12 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
 }
 
 // ============================================================ score pass helpers
+// Share of the score pass's rows split statically over the CTAs, and the
+// rows per dynamically handed-out chunk of the rest (CTAs that stream faster
+// take more of it; the counter is zeroed by k_prep).
+constexpr double kScoreStatic = 0.8;
+constexpr long long kScoreChunk = 1024;
+
 // The whole block searches the prefix in one round of loads: the unit
 // whose non-empty range [prefix[u], prefix[u+1]) holds x (0 if none).
 __device__ __forceinline__ int find_unit_block(const long long* prefix, int units, long long x, int* s_u) {
@@ -294,10 +301,15 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
   __syncthreads();
 
   const long long total = P.prefix[P.units];
-  const long long beg = total * blockIdx.x / gridDim.x;
-  const long long end = total * (blockIdx.x + 1) / gridDim.x;
-  if (beg >= end) return;
+  // static share in equal ranges, the rest in chunks from an atomic counter
+  const long long tstat = static_cast<long long>(static_cast<double>(total) * kScoreStatic);
+  const long long nchunk = (total - tstat + kScoreChunk - 1) / kScoreChunk;
   __shared__ int s_u;
+  __shared__ long long s_chunk;
+  long long beg = tstat * blockIdx.x / gridDim.x;
+  long long end = tstat * (blockIdx.x + 1) / gridDim.x;
+  for (;;) {
+  if (beg < end) {
   int u = find_unit_block(P.prefix, P.units, beg, &s_u);
   long long cur = beg;
   while (cur < end) {
@@ -338,6 +350,15 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
       flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
     }
     cur = uend;
+  }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt + 1, 1u));
+  __syncthreads();
+  const long long c = s_chunk;
+  if (c >= nchunk) break;
+  beg = tstat + c * kScoreChunk;
+  end = min(total, beg + kScoreChunk);
   }
 }
 
@@ -1325,15 +1346,22 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
   const T* cache = static_cast<const T*>(loki ? P.kp : P.k);
   const float* qsrc = loki ? P.qsel : P.qbar;
 
+  // work split: the first kScoreStatic of the rows in equal contiguous ranges
+  // per CTA, the rest in chunks of kScoreChunk rows handed out by an atomic
+  // counter (zeroed by k_prep), so CTAs that stream faster take more of it
   const long long total = P.prefix[P.units];
-  const long long beg = total * blockIdx.x / gridDim.x;
-  const long long end = total * (blockIdx.x + 1) / gridDim.x;
-  if (beg >= end) return;
+  const long long tstat = static_cast<long long>(static_cast<double>(total) * kScoreStatic);
+  const long long nchunk = (total - tstat + kScoreChunk - 1) / kScoreChunk;
   __shared__ int s_u;
-  int u = find_unit_block(P.prefix, P.units, beg, &s_u);
-  long long cur = beg;
+  __shared__ long long s_chunk;
   unsigned issued = 0;  // blocks this warp issued so far (stage and phase follow from it)
   bool failed = false;
+  long long beg = tstat * blockIdx.x / gridDim.x;
+  long long end = tstat * (blockIdx.x + 1) / gridDim.x;
+  for (;;) {
+  if (beg < end) {
+  int u = find_unit_block(P.prefix, P.units, beg, &s_u);
+  long long cur = beg;
   while (cur < end) {
     while (P.prefix[u + 1] <= cur) u++;
     const long long uend = min(end, P.prefix[u + 1]);
@@ -1406,6 +1434,16 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
       flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
     }
     cur = uend;
+  }
+  }
+  // next dynamic chunk
+  __syncthreads();
+  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt + 1, 1u));
+  __syncthreads();
+  const long long c = s_chunk;
+  if (c >= nchunk) break;
+  beg = tstat + c * kScoreChunk;
+  end = min(total, beg + kScoreChunk);
   }
 }
 
