@@ -43,7 +43,6 @@ struct vattn_ctx {
   unsigned* segcnt = nullptr;
   float* pscore = nullptr;
   long long* prefix = nullptr;
-  unsigned* cnt = nullptr;
   unsigned* gcnt = nullptr;
   long long* pre_det = nullptr;
   long long* pre_samp = nullptr;
@@ -233,7 +232,6 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   // only the grid-wide select reads the digit-2 and digit-3 histograms
   P->hist_words = (ctx->select1 || ctx->select_smem) ? vattn::kHist1 : vattn::kHistAll;
   P->prefix = ctx->prefix;
-  P->cnt = ctx->cnt;
   P->gcnt = ctx->gcnt;
   P->pre_det = ctx->pre_det;
   P->pre_samp = ctx->pre_samp;
@@ -346,13 +344,12 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const size_t sz_seg = align256(U * ctx->nseg * 2 * sizeof(unsigned));
   const size_t sz_ps = align256(U * cfg->max_ctx * G * sizeof(float));
   const size_t sz_pre = align256((U + 1) * sizeof(long long));
-  const size_t sz_cnt = align256(U * 2 * sizeof(unsigned));
   const size_t sz_gcnt = 256;
   const size_t sz_spre = align256((2 * U + 1) * sizeof(long long));
   const size_t sz_rdet = align256((ctx->CD + 2 * U) * REC * sizeof(float));
   const size_t sz_rsmp = align256((ctx->CS + 2 * U) * REC * sizeof(float));
   const size_t sz_err = 256;
-  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_pre + sz_cnt + sz_gcnt +
+  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_pre + sz_gcnt +
                   2 * sz_spre + sz_rdet + sz_rsmp + sz_err;
   if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -369,7 +366,6 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->segcnt = reinterpret_cast<unsigned*>(p); p += sz_seg;
   ctx->pscore = reinterpret_cast<float*>(p); p += sz_ps;
   ctx->prefix = reinterpret_cast<long long*>(p); p += sz_pre;
-  ctx->cnt = reinterpret_cast<unsigned*>(p); p += sz_cnt;
   ctx->gcnt = reinterpret_cast<unsigned*>(p); p += sz_gcnt;
   ctx->pre_det = reinterpret_cast<long long*>(p); p += sz_spre;
   ctx->pre_samp = reinterpret_cast<long long*>(p); p += sz_spre;

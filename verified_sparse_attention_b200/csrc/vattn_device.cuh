@@ -89,8 +89,7 @@ struct DevParams {
   float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
   int hist_words;   // histogram words per unit that k_prep zeroes (all only for the grid-wide select)
   long long* prefix;// [units + 1]: score-pass work prefix
-  unsigned* cnt;    // [units][2]: finished-segment counters of the det and sample gathers
-  unsigned* gcnt;   // finished-CTA counter of the det gather
+  unsigned* gcnt;   // [0]: score-pass chunks handed out (zeroed by k_prep)
   long long* pre_det;   // [2 units + 1]: slice prefix of the det (or dense) gather
   long long* pre_samp;  // [2 units + 1]: slice prefix of the sample gather
   float* rec_det;   // [CD + 2 units][G][2 + D]: det (or dense) gather records
@@ -158,26 +157,17 @@ __device__ __forceinline__ float chunk_dot(const float* q, const uint4& raw) {
   return acc;
 }
 
-// Chunk sums of one row live in the L lanes of an aligned lane group (lane li
-// holds chunk li). The row's dot is the halving-stride tree over chunks:
-// chunk l += chunk l + L/2, then l += l + L/4, ..., l += l + 1. A butterfly
-// with xor offsets L/2, ..., 1 produces exactly these sums in every lane
-// (each stage adds the same two operands, and fp addition is commutative).
-template <int L>
-__device__ __forceinline__ float group_allreduce(float v) {
-#pragma unroll
-  for (int o = L / 2; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
 __host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
 
-// The same tree for U rows at once (U <= L): at the first log2(U) stages each
-// lane keeps half of its rows and receives its partner's partials for them,
-// so U rows cost (U - 1) + log2(L/U) shuffles instead of U*log2(L). Each stage
-// still adds the partials of lanes x and x^o for a row, so every row's sum is
-// the same tree as group_allreduce. Afterwards the lanes
-// [r*(L/U), (r+1)*(L/U)) of the group hold row r.
+// Chunk sums of U rows live in the L lanes of an aligned lane group (lane li
+// holds chunk li of every row). Each row's dot is the halving-stride tree over
+// chunks: chunk l += chunk l + L/2, then l += l + L/4, ..., l += l + 1. At the
+// first log2(U) stages each lane keeps half of its rows and receives its
+// partner's partials for them, so U rows cost (U - 1) + log2(L/U) shuffles
+// instead of U*log2(L); every stage still adds the partials of lanes x and
+// x^o for a row (fp addition is commutative), so each row's sum is exactly
+// that tree. Afterwards the lanes [r*(L/U), (r+1)*(L/U)) of the group hold
+// row r (U <= L).
 template <int L, int U>
 __device__ __forceinline__ float reduce_rows(float (&a)[U], int li) {
   constexpr int LOGL = ilog2c(L);

@@ -148,7 +148,6 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
     if (tid == 0) {
       P.pre_det[ns] = carry;
       P.gcnt[0] = 0u;
-      P.gcnt[1] = 0u;
     }
     return;
   }
@@ -241,7 +240,6 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
 
   unsigned* hist = P.hist + static_cast<size_t>(u) * kHistAll;
   for (int i = tid; i < P.hist_words; i += blockDim.x) hist[i] = 0u;
-  if (tid < 2) P.cnt[2 * u + tid] = 0u;
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
   for (int i = tid; i < r.s1; i += blockDim.x) sel[i] = i;
   for (int i = tid; i < n - r.wst; i += blockDim.x) sel[r.s1 + r.k + i] = r.wst + i;
@@ -353,7 +351,7 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
   }
   }
   __syncthreads();
-  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt + 1, 1u));
+  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt, 1u));
   __syncthreads();
   const long long c = s_chunk;
   if (c >= nchunk) break;
@@ -1438,7 +1436,7 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
   }
   // next dynamic chunk
   __syncthreads();
-  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt + 1, 1u));
+  if (threadIdx.x == 0) s_chunk = static_cast<long long>(atomicAdd(P.gcnt, 1u));
   __syncthreads();
   const long long c = s_chunk;
   if (c >= nchunk) break;
@@ -2047,11 +2045,19 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
 // Positions of sampled entries. PHASE 0: the pilot draws (or the whole tail
 // when it is no larger than the pilot), after the cluster or grid-wide top-k
 // selection (k_select1 does this itself). PHASE 1, after the budget: draws t
-// in [p, b), or the whole tail when the budget covers it. Grid (units, splits).
+// in [p, b), or the whole tail when the budget covers it; CTA (0, 0) also
+// writes the sample gather's slice prefix (every budget is known by now).
+// Grid (units, splits).
 template <int PHASE>
 __global__ void __launch_bounds__(128) k_draws(DevParams P) {
   __shared__ int s_topk[kTopkSmem];
   grid_dependency_wait();
+  if (PHASE == 1 && blockIdx.x == 0 && blockIdx.y == 0) {
+    __shared__ unsigned s_warp[32];
+    __shared__ long long s_carry;
+    write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
+    __syncthreads();
+  }
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
   int t0 = 0, t1 = 0;
@@ -2073,30 +2079,15 @@ __global__ void __launch_bounds__(128) k_draws(DevParams P) {
 // ============================================================ k_budget
 // One CTA per unit: the per-head CLT budget from the det gather's records
 // (score maxima) and true scores.
-// The grid's last CTA to finish writes the sample gather's slice prefix (the
-// arrival counter is zeroed by k_prep).
 constexpr int kBudgetThreads = 512;
 template <int D, int G>
 __global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
   __shared__ float s_mh[G];
-  __shared__ unsigned s_warp[32];
-  __shared__ long long s_carry;
-  __shared__ bool s_last;
   grid_dependency_wait();
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
   if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
   unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();  // this unit's state before the arrival
-    s_last = atomicAdd(P.gcnt, 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
-  }
   grid_dependents_launch();
 }
 
