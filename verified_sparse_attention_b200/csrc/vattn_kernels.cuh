@@ -247,10 +247,10 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
 
 // ============================================================ score pass helpers
 // Share of the score pass's rows split statically over the CTAs, and the
-// rows per dynamically handed-out chunk of the rest (CTAs that stream faster
-// take more of it; the counter is zeroed by k_prep).
+// bytes of rows per dynamically handed-out chunk of the rest (CTAs that
+// stream faster take more of it; the counter is zeroed by k_prep).
 constexpr double kScoreStatic = 0.8;
-constexpr long long kScoreChunk = 1024;
+constexpr long long kScoreChunkBytes = 262144;
 
 // The whole block searches the prefix in one round of loads: the unit
 // whose non-empty range [prefix[u], prefix[u+1]) holds x (0 if none).
@@ -301,7 +301,8 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
   const long long total = P.prefix[P.units];
   // static share in equal ranges, the rest in chunks from an atomic counter
   const long long tstat = static_cast<long long>(static_cast<double>(total) * kScoreStatic);
-  const long long nchunk = (total - tstat + kScoreChunk - 1) / kScoreChunk;
+  constexpr long long kChunk = kScoreChunkBytes / (W * static_cast<long long>(sizeof(T)));
+  const long long nchunk = (total - tstat + kChunk - 1) / kChunk;
   __shared__ int s_u;
   __shared__ long long s_chunk;
   long long beg = tstat * blockIdx.x / gridDim.x;
@@ -355,8 +356,8 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
   __syncthreads();
   const long long c = s_chunk;
   if (c >= nchunk) break;
-  beg = tstat + c * kScoreChunk;
-  end = min(total, beg + kScoreChunk);
+  beg = tstat + c * kChunk;
+  end = min(total, beg + kChunk);
   }
 }
 
@@ -1345,11 +1346,12 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
   const float* qsrc = loki ? P.qsel : P.qbar;
 
   // work split: the first kScoreStatic of the rows in equal contiguous ranges
-  // per CTA, the rest in chunks of kScoreChunk rows handed out by an atomic
+  // per CTA, the rest in chunks of kScoreChunkBytes handed out by an atomic
   // counter (zeroed by k_prep), so CTAs that stream faster take more of it
   const long long total = P.prefix[P.units];
   const long long tstat = static_cast<long long>(static_cast<double>(total) * kScoreStatic);
-  const long long nchunk = (total - tstat + kScoreChunk - 1) / kScoreChunk;
+  constexpr long long kChunk = kScoreChunkBytes / (W * static_cast<long long>(sizeof(T)));
+  const long long nchunk = (total - tstat + kChunk - 1) / kChunk;
   __shared__ int s_u;
   __shared__ long long s_chunk;
   unsigned issued = 0;  // blocks this warp issued so far (stage and phase follow from it)
@@ -1440,8 +1442,8 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
   __syncthreads();
   const long long c = s_chunk;
   if (c >= nchunk) break;
-  beg = tstat + c * kScoreChunk;
-  end = min(total, beg + kScoreChunk);
+  beg = tstat + c * kChunk;
+  end = min(total, beg + kChunk);
   }
 }
 
