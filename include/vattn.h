@@ -23,8 +23,11 @@
  *
  * Memory: every array argument is caller-owned DEVICE memory unless stated;
  * the context owns only its workspace, allocated once in vattn_create.
- * vattn_decode allocates nothing, never synchronises the host, and enqueues
- * all its work on `stream`, so it may be captured in a CUDA graph.
+ * vattn_decode allocates no device memory, encodes two row maps of the K and
+ * V caches on the host (tensor-map descriptors, passed to the gathers by
+ * value), never synchronises the host, and enqueues all its work on
+ * `stream`, so it may be captured in a CUDA graph (score-pass timing, when
+ * enabled, adds event records on `stream`).
  *
  * Layouts (row-major, innermost last; Hq query heads, Hkv KV heads, d head
  * dim, G = Hq/Hkv, query head hq belongs to KV head hq / G):
@@ -107,7 +110,8 @@ typedef struct {
   float eps;         /* > 0: relative error target on the softmax denominator   */
   float delta;       /* in (0, 1): allowed failure probability                  */
   uint64_t seed;     /* Philox4x32-10 key of the tail sampler                   */
-  int num_pages;     /* pages in the caches (bound for page_table entries)      */
+  int num_pages;     /* pages in the caches (bound for page_table entries);     */
+                     /* num_pages * Hkv * page_size must stay below 2^31        */
   const void* k_t_cache;    /* SparQ: dim-major K [num_pages][Hkv][d][page_size], else NULL  */
   const void* k_proj_cache; /* Loki: projected K [num_pages][Hkv][page_size][rank], else NULL */
   const float* proj_basis;  /* Loki: basis fp32 [Hkv][d][rank], else NULL                     */
