@@ -1215,7 +1215,7 @@ __device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
 // otherwise). Block of kCombGroups * D threads: thread (r, e) folds every
 // kCombGroups-th record of each list with a running maximum (batches of
 // loads issued ahead of the fold), and the groups' states are then merged.
-constexpr int kCombGroups = 4;
+constexpr int kCombGroups = 8;
 
 template <int D, int G, int MODE>
 __device__ void unit_combine(const DevParams& P, int u, int g) {
