@@ -1983,7 +1983,7 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
     // lowest positions) and where its selections go.
     int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
     const bool stage = inf.k <= kTopkSmem;
-    unsigned taken = 0, eq_seen = 0;
+    unsigned gt_seen = 0, eq_seen = 0;
     __shared__ unsigned s_round[2];
     for (int base = 0; base < mlen; base += 32 * kSel1Threads) {
       const int wb = base + warp * 1024;
@@ -1999,18 +1999,21 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
           weq = be;
         }
       }
-      const unsigned ne = __popc(weq);
-      const unsigned eq_incl = block_inclusive_scan(ne, s_warp);
-      const unsigned eq_before = eq_seen + eq_incl - ne;
+      // one scan of (above, tied) counts packed in 16-bit halves (a round
+      // holds at most 32768 keys): a word's selections start at
+      // above_before + min(tied_before, need_eq), and it keeps its lowest
+      // need_eq - tied_before tied positions
+      const unsigned ng = __popc(wgt), ne = __popc(weq);
+      const unsigned incl = block_inclusive_scan((ng << 16) | ne, s_warp);
+      const unsigned excl = incl - ((ng << 16) | ne);
+      const unsigned gt_before = gt_seen + (excl >> 16), eq_before = eq_seen + (excl & 0xFFFFu);
       const unsigned keep = need_eq > eq_before ? min(ne, need_eq - eq_before) : 0u;
       unsigned wsel = wgt, e = weq;
       for (unsigned c = 0; c < keep; c++) {  // the lowest `keep` tied positions
         wsel |= e & (0u - e);
         e &= e - 1u;
       }
-      const unsigned nt = __popc(wsel);
-      const unsigned t_incl = block_inclusive_scan(nt, s_warp);
-      unsigned pos = taken + t_incl - nt;
+      unsigned pos = gt_before + min(eq_before, need_eq);
       while (wsel) {
         const int j = inf.s1 + wb + lane * 32 + (__ffs(wsel) - 1);
         sel[pos] = j;
@@ -2019,12 +2022,12 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
         wsel &= wsel - 1u;
       }
       if (tid == kSel1Threads - 1) {  // round totals: the last thread holds the inclusive sums
-        s_round[0] = eq_incl;
-        s_round[1] = t_incl;
+        s_round[0] = incl & 0xFFFFu;
+        s_round[1] = incl >> 16;
       }
       __syncthreads();
       eq_seen += s_round[0];
-      taken += s_round[1];
+      gt_seen += s_round[1];
       __syncthreads();
     }
     __syncthreads();  // the staged list is complete
