@@ -16,6 +16,8 @@ from . import build as _build
 
 F32, BF16 = 0, 1
 EXACT, SPARQ, LOKI = 0, 1, 2
+GUARANTEE_DENOMINATOR, GUARANTEE_OUTPUT = 0, 1
+GUARANTEES = {"denominator": GUARANTEE_DENOMINATOR, "output": GUARANTEE_OUTPUT}
 DTYPES = {"f32": F32, "bf16": BF16}
 PROXIES = {"exact": EXACT, "sparq": SPARQ, "loki": LOKI}
 
@@ -30,6 +32,7 @@ class Problem(C.Structure):
         ("topk_abs", C.c_int), ("topk_num", C.c_int), ("topk_den", C.c_int),
         ("pilot_min", C.c_int), ("pilot_num", C.c_int), ("pilot_den", C.c_int),
         ("eps", C.c_float), ("delta", C.c_float), ("seed", C.c_uint64),
+        ("guarantee", C.c_int),
     ]
 
 
@@ -124,8 +127,11 @@ def ord_key(f, L=None):
     return (L or lib()).orc_ord(float(f))
 
 
-def make_problem(w, seed=None, eps=None, batch=None):
-    """Problem struct from a workload description (verified_sparse_attention_b200.synth.Workload)."""
+def make_problem(w, seed=None, eps=None, batch=None, guarantee=None):
+    """Problem struct from a workload description (verified_sparse_attention_b200.synth.Workload).
+
+    `guarantee` ("denominator" or "output") overrides the workload's own.
+    """
     return Problem(
         batch=batch if batch is not None else w.batch, num_q_heads=w.num_q_heads,
         num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, dtype=DTYPES[w.dtype],
@@ -134,7 +140,8 @@ def make_problem(w, seed=None, eps=None, batch=None):
         topk_abs=w.topk_abs, topk_num=w.topk_num, topk_den=w.topk_den,
         pilot_min=w.pilot_min, pilot_num=w.pilot_num, pilot_den=w.pilot_den,
         eps=w.eps if eps is None else eps, delta=w.delta,
-        seed=w.seed if seed is None else seed)
+        seed=w.seed if seed is None else seed,
+        guarantee=GUARANTEES[guarantee or getattr(w, "guarantee", "denominator")])
 
 
 def decode(problem, inputs, units=None, L=None):

@@ -15,7 +15,9 @@
  *        uniform random sample of the remaining indices, whose size is chosen
  *        from the Central Limit Theorem so that the user's (eps, delta) accuracy
  *        holds; the paragraph after it says the guarantee is placed on the
- *        softmax denominator.
+ *        softmax denominator, calling that a relaxation of guaranteeing the
+ *        attention output (the numerator as well) which makes the budget
+ *        cheaper to compute. The unrelaxed form is the output guarantee here.
  *   [SQ] "SparQ Attention: Bandwidth-Efficient LLM Inference", abstract:
  *        approximate scores from selectively fetched parts of the cache.
  *   [LK] "Loki: Low-rank Keys for Efficient Sparse Attention", abstract: rank
@@ -45,6 +47,9 @@
 #define ORC_SPARQ 1
 #define ORC_LOKI 2
 
+#define ORC_GUARANTEE_DENOMINATOR 0
+#define ORC_GUARANTEE_OUTPUT 1
+
 typedef unsigned __int128 u128;
 
 typedef struct {
@@ -56,6 +61,7 @@ typedef struct {
   int pilot_min, pilot_num, pilot_den;
   float eps, delta;
   uint64_t seed;
+  int guarantee; /* ORC_GUARANTEE_DENOMINATOR or ORC_GUARANTEE_OUTPUT */
 } orc_problem;
 
 /* ------------------------------------------------------------------ */
@@ -390,6 +396,8 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
     }
     float* sf = malloc(sizeof(float) * (size_t)nI);
     float* sp = malloc(sizeof(float) * (size_t)p);
+    float* xf = malloc(sizeof(float) * (size_t)nI);
+    float* xp = malloc(sizeof(float) * (size_t)p);
     int nmax = 0;
     for (int g = 0; g < G; g++) {
       const float* qg = qh + (size_t)g * d;
@@ -406,10 +414,12 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
       u128 S2 = 0;
       for (int i = 0; i < nI; i++) {
         float x = orc_vexp(sf[i] - m);
+        xf[i] = x;
         Sf += (uint64_t)llrintf(x * 4294967296.0f);
       }
       for (int t = 0; t < p; t++) {
         float x = orc_vexp(sp[t] - m);
+        xp[t] = x;
         uint64_t xq = (uint64_t)llrintf(x * 4294967296.0f);
         S1 += xq;
         S2 += (u128)xq * xq;
@@ -421,6 +431,50 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
       double t = (z * (double)ntail) / ((double)pr->eps * Dq);
       double need = (t * t) * var;
       int nh = need >= (double)ntail ? ntail : (int)ceil(need);
+      if (pr->guarantee == ORC_GUARANTEE_OUTPUT) {
+        /* Output guarantee (reading: the pages state only that the         */
+        /* denominator-only budget relaxes it). The same CLT condition is   */
+        /* put on the numerator vector Nv = sum_j x_j v_j: estimated from   */
+        /* b tail draws, its error has covariance N_tail^2 Sigma / b with   */
+        /* Sigma the covariance of x v over the tail, so its expected       */
+        /* squared length is N_tail^2 tr(Sigma) / b, and                    */
+        /*   n >= (z * N_tail / (eps * |Nv|))^2 * tr(Sigma),                */
+        /* tr(Sigma) = sum over dims of the unbiased pilot variance of x v, */
+        /* |Nv| = length of (sum over I_f of x v) + N_tail * (pilot mean).  */
+        /* In double: each product x * v is exact (24 x 24 significant      */
+        /* bits at most); sums run over I_f in list order and over the      */
+        /* pilot in draw order, then over dims ascending. A negative        */
+        /* variance (rounding) counts as 0; |Nv| = 0 takes the whole tail   */
+        /* unless every variance is 0 as well.                              */
+        double tr = 0.0, nsq = 0.0;
+        for (int e = 0; e < d; e++) {
+          double A = 0.0, T1 = 0.0, T2 = 0.0;
+          for (int i = 0; i < nI; i++)
+            A = A + (double)xf[i] * (double)elem(in->v_cache, row_base(pr, in->page_table, b, h, If[i], d) + e, dt);
+          for (int t = 0; t < p; t++) {
+            double y = (double)xp[t] * (double)elem(in->v_cache, row_base(pr, in->page_table, b, h, pil[t], d) + e, dt);
+            T1 = T1 + y;
+            T2 = T2 + y * y;
+          }
+          double ve = ((double)p * T2 - T1 * T1) / ((double)p * (double)(p - 1));
+          if (ve < 0.0) ve = 0.0;
+          double Ne = A + ((double)ntail * T1) / (double)p;
+          tr = tr + ve;
+          nsq = nsq + Ne * Ne;
+        }
+        /* the pilot mean's own noise adds N_tail^2 tr(Sigma) / p to |Nv|^2 */
+        /* in expectation; it is taken off (unbiased estimate of |Nv|^2)    */
+        double nsq_u = nsq - (((double)ntail * (double)ntail) / (double)p) * tr;
+        double need_v;
+        if (nsq_u > 0.0) {
+          double tv = (z * (double)ntail) / ((double)pr->eps * sqrt(nsq_u));
+          need_v = (tv * tv) * tr;
+        } else {
+          need_v = tr > 0.0 ? (double)ntail : 0.0;
+        }
+        int nv = need_v >= (double)ntail ? ntail : (int)ceil(need_v);
+        if (nv > nh) nh = nv;
+      }
       need_h[g] = nh;
       if (nh > nmax) nmax = nh;
     }
@@ -432,6 +486,8 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
     free(pil);
     free(sf);
     free(sp);
+    free(xf);
+    free(xp);
   }
 
   /* Selected list: I_f, then the b draws in draw order (the pilot is the    */
@@ -513,6 +569,7 @@ int orc_decode(const orc_problem* pr, const void* q, const void* k_cache, const 
   if (G & (G - 1)) return -1;
   if (!(pr->eps > 0.0f) || !(pr->delta > 0.0f && pr->delta < 1.0f)) return -1;
   if (pr->pilot_min < 2) return -1;
+  if (pr->guarantee != ORC_GUARANTEE_DENOMINATOR && pr->guarantee != ORC_GUARANTEE_OUTPUT) return -1;
   if (pr->sinks < 0 || pr->window < 0 || pr->topk_abs < 0 || pr->topk_num < 0 || pr->topk_den < 0 ||
       pr->pilot_num < 0 || pr->pilot_den < 0)
     return -1;

@@ -58,6 +58,7 @@ class Workload:
     seed: int               # sampler seed
     data_seed: int
     recipe: str
+    guarantee: str = "denominator"  # "denominator" | "output": what the budget bounds
 
     @property
     def pages_per_seq(self):
