@@ -1,6 +1,7 @@
 """Benchmark of the verified sparse decode step (vattn_decode) on B200.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload gqa_32k] [--eps E]
+                    [--guarantee denominator|output]
     python bench.py --impl reference ...      # the CPU oracle, timed on host cores
 
 One step = one vattn_decode call over the whole batch of the workload (every
@@ -132,6 +133,16 @@ def algorithmic_bytes(w, x, res):
     score = int(mid.sum()) * w.num_kv_heads * (per_row + 4)     # K (or proxy) read + key write
     cnt = res["sel_count"].to(torch.int64).cpu()            # [B, Hkv] rows gathered (K and V)
     gather = int(cnt.sum()) * 2 * d * e
+    if w.guarantee == "output":
+        # the numerator statistics read the V rows of I_f and the pilot once more
+        # for every unit that drew a pilot (N_tail > p)
+        kb = (n * w.topk_num) // w.topk_den if w.topk_den else torch.full_like(n, w.topk_abs)
+        k = torch.minimum(kb, mid)
+        p = (torch.clamp((n * w.pilot_num + w.pilot_den - 1) // w.pilot_den, min=w.pilot_min)
+             if w.pilot_den else torch.full_like(n, w.pilot_min))
+        n_if = s1 + k + (n - wst)
+        piloted = (mid - k) > p
+        gather += int(((n_if + p) * piloted).sum()) * w.num_kv_heads * d * e
     return score, score + gather
 
 
@@ -139,7 +150,7 @@ def algorithmic_bytes(w, x, res):
 def run_gpu_arm(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[args.workload].replace(guarantee=args.guarantee)
     w = ranks.rank_workload(w, rank)
     x = synth.make_inputs(w, device=dev)
     dec = decoder_for(w, device=dev)
@@ -307,6 +318,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gqa_32k", choices=list(synth.WORKLOADS))
     ap.add_argument("--eps", type=float, default=None)
+    ap.add_argument("--guarantee", default="denominator", choices=["denominator", "output"],
+                    help="what the sample size bounds: the softmax denominator, or the output too")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -315,7 +328,7 @@ def main():
         ap.error("--warmup must be >= 3")
 
     world, rank, local_rank = ranks.rank_env()
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[args.workload].replace(guarantee=args.guarantee)
     if args.eps is not None:
         w = w.replace(eps=args.eps)
     cfg = {"workload": synth.describe(w), "name": w.name, "batch": w.batch,

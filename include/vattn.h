@@ -16,6 +16,15 @@
  *     probability about 1 - delta;
  *   - output o = (A_f + (N_tail/b) A_s) / (L_f + (N_tail/b) L_s), where A and
  *     L are the exp-weighted value sums and exp sums over I_f and the sample.
+ * The same page calls the denominator-only bound a relaxation of bounding the
+ * attention output. With vattn_params.guarantee = VATTN_GUARANTEE_OUTPUT the
+ * budget also bounds the numerator vector Nv = sum_j x_j v_j (x_j =
+ * exp(s_j - m)) by the same CLT condition (a reading; the pages give no
+ * formula): n >= (z * N_tail / (eps * |Nv|))^2 * tr(Sigma), with tr(Sigma)
+ * the sum over dimensions of the pilot's unbiased variance of x v, and |Nv|^2
+ * the pilot's unbiased estimate (|Nv_hat|^2 - N_tail^2 tr(Sigma) / p; not
+ * positive: the whole tail). Computed in double in a fixed order (items in
+ * list order, then dimensions ascending), so it is reproducible bit for bit.
  * The ranking score is exact (q . k), a SparQ-style proxy over the r largest
  * query components ("SparQ Attention: Bandwidth-Efficient LLM Inference",
  * abstract), or a Loki-style score in a stored low-rank key space ("Loki:
@@ -68,6 +77,9 @@ extern "C" {
 
 enum { VATTN_FP32 = 0, VATTN_BF16 = 1 };
 enum { VATTN_EXACT = 0, VATTN_SPARQ = 1, VATTN_LOKI = 2 };
+/* what the sample size bounds: the softmax denominator alone (the pages'
+   practical form), or the denominator and the numerator vector (output) */
+enum { VATTN_GUARANTEE_DENOMINATOR = 0, VATTN_GUARANTEE_OUTPUT = 1 };
 
 enum {
   VATTN_OK = 0,
@@ -108,6 +120,7 @@ typedef struct {
      max(pilot_min, ceil(N * pilot_num / pilot_den)); pilot_min >= 2           */
   int pilot_min, pilot_num, pilot_den;
   float eps;         /* > 0: relative error target on the softmax denominator   */
+                     /* (and on |Nv| with the output guarantee)                  */
   float delta;       /* in (0, 1): allowed failure probability                  */
   uint64_t seed;     /* Philox4x32-10 key of the tail sampler                   */
   int num_pages;     /* pages in the caches (bound for page_table entries);     */
@@ -115,6 +128,9 @@ typedef struct {
   const void* k_t_cache;    /* SparQ: dim-major K [num_pages][Hkv][d][page_size], else NULL  */
   const void* k_proj_cache; /* Loki: projected K [num_pages][Hkv][page_size][rank], else NULL */
   const float* proj_basis;  /* Loki: basis fp32 [Hkv][d][rank], else NULL                     */
+  int guarantee;     /* VATTN_GUARANTEE_DENOMINATOR (0) or VATTN_GUARANTEE_OUTPUT;  */
+                     /* OUTPUT adds one kernel that reads the V rows of I_f and the */
+                     /* pilot once more; anything else: VATTN_EINVAL                */
 } vattn_params;
 
 /* Create a context on the current CUDA device and allocate its workspace.

@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libvattn.so")
 
 VATTN_FP32, VATTN_BF16 = 0, 1
 VATTN_EXACT, VATTN_SPARQ, VATTN_LOKI = 0, 1, 2
+VATTN_GUARANTEE_DENOMINATOR, VATTN_GUARANTEE_OUTPUT = 0, 1
 VATTN_OK, VATTN_EINVAL, VATTN_ENOMEM, VATTN_ECUDA, VATTN_ESCRATCH = 0, -1, -2, -3, -4
 VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE, VATTN_DEV_TIMEOUT = 1, 2, 4
 
@@ -35,7 +36,8 @@ class vattn_params(C.Structure):
                 ("pilot_min", C.c_int), ("pilot_num", C.c_int), ("pilot_den", C.c_int),
                 ("eps", C.c_float), ("delta", C.c_float), ("seed", C.c_uint64),
                 ("num_pages", C.c_int),
-                ("k_t_cache", C.c_void_p), ("k_proj_cache", C.c_void_p), ("proj_basis", C.c_void_p)]
+                ("k_t_cache", C.c_void_p), ("k_proj_cache", C.c_void_p), ("proj_basis", C.c_void_p),
+                ("guarantee", C.c_int)]
 
 
 class VattnError(RuntimeError):

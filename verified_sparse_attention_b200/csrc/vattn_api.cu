@@ -42,6 +42,7 @@ struct vattn_ctx {
   unsigned* hist = nullptr;
   unsigned* segcnt = nullptr;
   float* pscore = nullptr;
+  int* num_need = nullptr;
   long long* prefix = nullptr;
   unsigned* gcnt = nullptr;
   long long* pre_det = nullptr;
@@ -135,6 +136,7 @@ struct Kernels {
   void (*sample)(DevParams);
   void (*dense)(DevParams);
   void (*budget)(DevParams);
+  void (*numstats)(DevParams);
   void (*combine_sample)(DevParams);
   void (*combine_dense)(DevParams);
   size_t gather_smem;
@@ -156,6 +158,7 @@ Kernels kernels_for() {
   k.sample = vattn::k_gather<T, D, G, vattn::kModeSample>;
   k.dense = vattn::k_gather<T, D, G, vattn::kModeDense>;
   k.budget = vattn::k_budget<D, G>;
+  k.numstats = vattn::k_numstats<T, D, G>;
   k.combine_sample = vattn::k_combine<D, G, vattn::kModeSample>;
   k.combine_dense = vattn::k_combine<D, G, vattn::kModeDense>;
   k.gather_smem = vattn::GatherShape<T, D, G>::SMEM;
@@ -229,6 +232,7 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->hist = ctx->hist;
   P->segcnt = ctx->segcnt;
   P->pscore = ctx->pscore;
+  P->num_need = ctx->num_need;
   // only the grid-wide select reads the digit-2 and digit-3 histograms
   P->hist_words = (ctx->select1 || ctx->select_smem) ? vattn::kHist1 : vattn::kHistAll;
   P->prefix = ctx->prefix;
@@ -325,6 +329,7 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->gather_threads = K.gather_threads;
   for (auto fn : {K.det, K.sample, K.dense})
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->gather_smem));
+  cudaFuncSetAttribute(K.numstats, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(vattn::kNumSmem));
   int gocc = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, K.gather_threads, ctx->gather_smem);
   if (gocc < 1) gocc = 1;
@@ -343,13 +348,14 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const size_t sz_hist = align256(U * vattn::kHistAll * sizeof(unsigned));
   const size_t sz_seg = align256(U * ctx->nseg * 2 * sizeof(unsigned));
   const size_t sz_ps = align256(U * cfg->max_ctx * G * sizeof(float));
+  const size_t sz_nneed = align256(U * G * sizeof(int));
   const size_t sz_pre = align256((U + 1) * sizeof(long long));
   const size_t sz_gcnt = 256;
   const size_t sz_spre = align256((2 * U + 1) * sizeof(long long));
   const size_t sz_rdet = align256((ctx->CD + 2 * U) * REC * sizeof(float));
   const size_t sz_rsmp = align256((ctx->CS + 2 * U) * REC * sizeof(float));
   const size_t sz_err = 256;
-  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_pre + sz_gcnt +
+  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_nneed + sz_pre + sz_gcnt +
                   2 * sz_spre + sz_rdet + sz_rsmp + sz_err;
   if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -365,6 +371,7 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->hist = reinterpret_cast<unsigned*>(p); p += sz_hist;
   ctx->segcnt = reinterpret_cast<unsigned*>(p); p += sz_seg;
   ctx->pscore = reinterpret_cast<float*>(p); p += sz_ps;
+  ctx->num_need = reinterpret_cast<int*>(p); p += sz_nneed;
   ctx->prefix = reinterpret_cast<long long*>(p); p += sz_pre;
   ctx->gcnt = reinterpret_cast<unsigned*>(p); p += sz_gcnt;
   ctx->pre_det = reinterpret_cast<long long*>(p); p += sz_spre;
@@ -464,6 +471,8 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   if (!(prm->eps > 0.0f) || !isfinite(prm->eps)) return VATTN_EINVAL;
   if (!(prm->delta > 0.0f && prm->delta < 1.0f)) return VATTN_EINVAL;
   if (prm->num_pages < 1) return VATTN_EINVAL;
+  if (prm->guarantee != VATTN_GUARANTEE_DENOMINATOR && prm->guarantee != VATTN_GUARANTEE_OUTPUT)
+    return VATTN_EINVAL;
   if (c.proxy == VATTN_SPARQ && (!prm->k_t_cache || !aligned16(prm->k_t_cache))) return VATTN_EINVAL;
   if (c.proxy == VATTN_LOKI && (!prm->k_proj_cache || !prm->proj_basis || !aligned16(prm->k_proj_cache)))
     return VATTN_EINVAL;
@@ -493,6 +502,7 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.z = ctx->cached_z;
   P.seed = prm->seed;
   P.num_pages = prm->num_pages;
+  P.guarantee = prm->guarantee == VATTN_GUARANTEE_OUTPUT;
   if (const int rc = encode_row_maps(c, k_cache, v_cache, prm->num_pages, &P)) return ctx->last_status = rc;
   P.q = q;
   P.k = k_cache;
@@ -548,6 +558,9 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(128), 0, st, P, &launches);
   }
   launch(K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  if (P.guarantee)
+    launch(K.numstats, dim3(P.units, (ctx->G * c.head_dim + vattn::kNumThreads - 1) / vattn::kNumThreads),
+           dim3(vattn::kNumThreads), vattn::kNumSmem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(vattn::kBudgetThreads), 0, st, P, &launches);
   launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(128), 0, st, P, &launches);
   launch(K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);

@@ -62,6 +62,7 @@ struct DevParams {
   double z;
   unsigned long long seed;
   int nseg, dense;
+  int guarantee;    // 1: the budget also bounds the numerator vector (output guarantee)
   int CD, CS;       // grid sizes of the det (and dense) and sample gathers
   // inputs
   const void* q;
@@ -87,6 +88,7 @@ struct DevParams {
   unsigned* hist;   // [units][kHistAll]
   unsigned* segcnt; // [units][nseg][2]
   float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
+  int* num_need;    // [units][G]: numerator sizes n_v (output guarantee)
   int hist_words;   // histogram words per unit that k_prep zeroes (all only for the grid-wide select)
   long long* prefix;// [units + 1]: score-pass work prefix
   unsigned* gcnt;   // [0]: score-pass chunks handed out (zeroed by k_prep)

@@ -1156,7 +1156,8 @@ __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, cons
     const double Dq = __dadd_rn(__ull2double_rn(Sf), __ddiv_rn(__dmul_rn(nt, __ull2double_rn(S1)), pd));
     const double t = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), Dq));
     const double need = __dmul_rn(__dmul_rn(t, t), var);
-    const int nh = need >= nt ? inf.ntail : static_cast<int>(ceil(need));
+    int nh = need >= nt ? inf.ntail : static_cast<int>(ceil(need));
+    if (P.guarantee) nh = max(nh, P.num_need[u * G + g]);
     s_need[g] = nh;
     P.head_need[static_cast<size_t>(b) * P.Hq + h * G + g] = nh;
   }
@@ -2093,6 +2094,158 @@ __global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
   const UnitInfo inf = P.info[u];
   if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
   unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
+  grid_dependents_launch();
+}
+
+// ============================================================ k_numstats
+// Output guarantee: the numerator part of each query head's budget, from the
+// pilot. Grid (units, ceil(G * D / kNumThreads)); thread t of CTA y serves
+// head g = (y * kNumThreads + t) / D, dimension e = (y * kNumThreads + t) % D.
+// Items are I_f (list order) then the pilot draws (draw order), with their
+// true scores s and x = vexp(s - m_h) as in the budget. In double, with each
+// product x * v exact (24 x 24 significant bits at most) and every sum in
+// item order:
+//   A = sum over I_f of x v_e;  T1, T2 = sums over the pilot of y, y * y, y = x v_e;
+//   var_e = max(0, (p T2 - T1^2) / (p (p - 1)));  Nv_e = A + N_tail T1 / p.
+// One thread per head then sums var_e and Nv_e^2 over e ascending into tr and
+// |Nv_hat|^2, takes off the pilot mean's own noise N_tail^2 tr / p, and writes
+//   n_v = (z N_tail / (eps |Nv|))^2 tr   (the whole tail when |Nv|^2 <= 0 < tr)
+// to num_need; k_budget takes max(n_h, n_v). The items' row indices are
+// looked up once per block of kNumOffItems items (one parallel pass over
+// sel and the page table); the V rows and the true scores of each round of
+// items then stream through a kNumStages-deep ring of shared-memory buffers
+// by cp.async copies, and x is computed once per (item, head) when a round
+// has landed.
+constexpr int kNumThreads = 128;
+constexpr int kNumBufBytes = 16384;
+constexpr int kNumStages = 3;
+constexpr int kNumOffItems = 4096;
+constexpr size_t kNumSmem = static_cast<size_t>(kNumStages) * kNumBufBytes + kNumOffItems * 4;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kNumThreads) k_numstats(DevParams P) {
+  constexpr int HPB = kNumThreads / D;                      // heads per CTA (1 or 2)
+  constexpr int ROWB = D * static_cast<int>(sizeof(T));     // bytes per V row
+  constexpr int CH = kNumBufBytes / ROWB;                   // items per round
+  constexpr int V16 = ROWB / 16;                            // 16-byte pieces per row
+  static_assert(kNumOffItems % CH == 0, "rounds must not straddle offset blocks");
+  extern __shared__ __align__(16) unsigned char num_smem[];
+  unsigned char* s_v = num_smem;                                                    // [stages][16 KB]
+  unsigned* s_row = reinterpret_cast<unsigned*>(num_smem + kNumStages * kNumBufBytes);  // [kNumOffItems]
+  __shared__ float s_ps[kNumStages][CH * G];  // true scores of a round, [item][head]
+  __shared__ double s_x[CH][HPB];
+  __shared__ float s_mh[G];
+  __shared__ double s_red[2][kNumThreads];
+  grid_dependency_wait();
+  const int u = blockIdx.x;
+  const UnitInfo inf = P.info[u];
+  if (inf.mode != 2) {
+    grid_dependents_launch();
+    return;
+  }
+  det_record_max<D, G>(P, u, s_mh);
+  const int b = u / P.Hkv, h = u % P.Hkv;
+  const int tid = threadIdx.x;
+  const int g0 = blockIdx.y * HPB;
+  const int hh = tid / D, e = tid % D;
+  const bool active = g0 + hh < G;
+  const int nA = inf.nI + inf.p;
+  const int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
+  const float* ps = P.pscore + static_cast<size_t>(u) * P.max_ctx * G;
+  const char* vb = static_cast<const char*>(P.v);
+  double A = 0.0, T1 = 0.0, T2 = 0.0;
+  for (int s0 = 0; s0 < nA; s0 += kNumOffItems) {
+    const int ns = min(kNumOffItems, nA - s0);
+    __syncthreads();  // the previous block's rounds are done with s_row and the ring
+#pragma unroll 4
+    for (int i = tid; i < ns; i += kNumThreads)
+      s_row[i] = static_cast<unsigned>(row_off(P, b, h, sel[s0 + i], 1));
+    __syncthreads();
+    const int rounds = (ns + CH - 1) / CH;
+    auto issue = [&](int r) {
+      const int c0 = r * CH, cnt = min(CH, ns - c0), buf = r % kNumStages;
+      unsigned char* dst = s_v + buf * kNumBufBytes;
+      for (int x = tid; x < cnt * V16; x += kNumThreads) {
+        const int i = x / V16, k = x % V16;
+        cp_async16(dst + i * ROWB + k * 16, vb + static_cast<size_t>(s_row[c0 + i]) * ROWB + k * 16);
+      }
+      const float* src = ps + static_cast<size_t>(s0 + c0) * G;
+      for (int x = tid; x < cnt * G; x += kNumThreads) cp_async4(&s_ps[buf][x], src + x);
+    };
+#pragma unroll
+    for (int r = 0; r < kNumStages - 1; r++) {
+      if (r < rounds) issue(r);
+      cp_async_commit();
+    }
+    for (int r = 0; r < rounds; r++) {
+      cp_async_wait<kNumStages - 2>();  // this thread's copies of round r have landed
+      __syncthreads();                  // everyone's have, and round r - 1 is consumed
+      if (r + kNumStages - 1 < rounds) issue(r + kNumStages - 1);
+      cp_async_commit();
+      const int c0 = r * CH, cnt = min(CH, ns - c0), buf = r % kNumStages;
+      for (int x = tid; x < cnt * HPB; x += kNumThreads) {
+        const int i = x / HPB, j = x % HPB;
+        const int g = min(g0 + j, G - 1);
+        s_x[i][j] = static_cast<double>(vexp(__fsub_rn(s_ps[buf][i * G + g], s_mh[g])));
+      }
+      __syncthreads();
+      if (active) {
+        const T* rows = reinterpret_cast<const T*>(s_v + buf * kNumBufBytes);
+        const int nIr = inf.nI - (s0 + c0);  // items [0, nIr) of this round are in I_f
+        // x * v is exact in double, so A + x * v rounded once (an FMA) is
+        // the same as the rounded sum of the exact product
+        const int nIc = max(0, min(cnt, nIr));
+#pragma unroll 4
+        for (int i = 0; i < nIc; i++)
+          A = __fma_rn(s_x[i][hh], static_cast<double>(Elem<T>::load(rows, static_cast<size_t>(i) * D + e)), A);
+#pragma unroll 4
+        for (int i = nIc; i < cnt; i++) {
+          const double y = __dmul_rn(s_x[i][hh], static_cast<double>(Elem<T>::load(rows, static_cast<size_t>(i) * D + e)));
+          T1 = __dadd_rn(T1, y);
+          T2 = __dadd_rn(T2, __dmul_rn(y, y));
+        }
+      }
+    }
+    cp_async_wait<0>();
+  }
+  const double pd = static_cast<double>(inf.p), nt = static_cast<double>(inf.ntail);
+  double ve = __ddiv_rn(__dsub_rn(__dmul_rn(pd, T2), __dmul_rn(T1, T1)),
+                        __dmul_rn(pd, static_cast<double>(inf.p - 1)));
+  if (ve < 0.0) ve = 0.0;
+  const double nv = __dadd_rn(A, __ddiv_rn(__dmul_rn(nt, T1), pd));
+  s_red[0][tid] = ve;
+  s_red[1][tid] = __dmul_rn(nv, nv);
+  __syncthreads();
+  if (tid < HPB && g0 + tid < G) {
+    double tr = 0.0, nsq = 0.0;
+    for (int k = 0; k < D; k++) {
+      tr = __dadd_rn(tr, s_red[0][tid * D + k]);
+      nsq = __dadd_rn(nsq, s_red[1][tid * D + k]);
+    }
+    const double nsq_u = __dsub_rn(nsq, __dmul_rn(__ddiv_rn(__dmul_rn(nt, nt), pd), tr));
+    double need;
+    if (nsq_u > 0.0) {
+      const double tv = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), __dsqrt_rn(nsq_u)));
+      need = __dmul_rn(__dmul_rn(tv, tv), tr);
+    } else {
+      need = tr > 0.0 ? nt : 0.0;
+    }
+    P.num_need[u * G + g0 + tid] = need >= nt ? inf.ntail : static_cast<int>(ceil(need));
+  }
   grid_dependents_launch();
 }
 

@@ -9,6 +9,7 @@ from . import _abi
 
 _DTYPES = {torch.float32: _abi.VATTN_FP32, torch.bfloat16: _abi.VATTN_BF16}
 _PROXIES = {"exact": _abi.VATTN_EXACT, "sparq": _abi.VATTN_SPARQ, "loki": _abi.VATTN_LOKI}
+_GUARANTEES = {"denominator": _abi.VATTN_GUARANTEE_DENOMINATOR, "output": _abi.VATTN_GUARANTEE_OUTPUT}
 
 
 class SparseDecoder:
@@ -40,14 +41,15 @@ class SparseDecoder:
     @staticmethod
     def make_params(*, sinks, window, topk_abs=0, topk_num=0, topk_den=0, pilot_min=64,
                     pilot_num=0, pilot_den=0, eps, delta, seed, num_pages, k_t_cache=None,
-                    k_proj_cache=None, proj_basis=None):
+                    k_proj_cache=None, proj_basis=None, guarantee="denominator"):
         return _abi.vattn_params(
             sinks=sinks, window=window, topk_abs=topk_abs, topk_num=topk_num, topk_den=topk_den,
             pilot_min=pilot_min, pilot_num=pilot_num, pilot_den=pilot_den, eps=eps, delta=delta,
             seed=seed, num_pages=num_pages,
             k_t_cache=None if k_t_cache is None else k_t_cache.data_ptr(),
             k_proj_cache=None if k_proj_cache is None else k_proj_cache.data_ptr(),
-            proj_basis=None if proj_basis is None else proj_basis.data_ptr())
+            proj_basis=None if proj_basis is None else proj_basis.data_ptr(),
+            guarantee=_GUARANTEES[guarantee])
 
     def decode(self, q, k_cache, v_cache, page_table, seq_lens, params, outputs=None, stream=None):
         batch = q.shape[0]
@@ -90,11 +92,12 @@ def decoder_for(w, device=None, max_batch=None):
                          proxy=w.proxy, proxy_rank=w.proxy_rank, device=device)
 
 
-def params_for(w, inputs, eps=None, seed=None):
+def params_for(w, inputs, eps=None, seed=None, guarantee=None):
     """vattn_params of a synthetic workload with its drawn inputs (device tensors)."""
     return SparseDecoder.make_params(
         sinks=w.sinks, window=w.window, topk_abs=w.topk_abs, topk_num=w.topk_num,
         topk_den=w.topk_den, pilot_min=w.pilot_min, pilot_num=w.pilot_num, pilot_den=w.pilot_den,
         eps=w.eps if eps is None else eps, delta=w.delta, seed=w.seed if seed is None else seed,
         num_pages=int(inputs["num_pages"]), k_t_cache=inputs.get("k_t_cache"),
-        k_proj_cache=inputs.get("k_proj_cache"), proj_basis=inputs.get("proj_basis"))
+        k_proj_cache=inputs.get("k_proj_cache"), proj_basis=inputs.get("proj_basis"),
+        guarantee=guarantee or w.guarantee)

@@ -216,7 +216,8 @@ def describe(w):
     return (f"{w.name}: B{w.batch} Hq{w.num_q_heads}/Hkv{w.num_kv_heads} d{w.head_dim} {w.dtype} "
             f"N={'%d' % w.max_ctx if w.min_ctx == w.max_ctx else '%d..%d' % (w.min_ctx, w.max_ctx)} "
             f"ps{w.page_size} {w.proxy}{'' if w.proxy == 'exact' else ' r%d' % w.proxy_rank} "
-            f"s{w.sinks} w{w.window} eps{w.eps} delta{w.delta}")
+            f"s{w.sinks} w{w.window} eps{w.eps} delta{w.delta}"
+            + ("" if w.guarantee == "denominator" else f" guarantee={w.guarantee}"))
 
 
 __all__ = ["Workload", "WORKLOADS", "PAGED_EPS_SWEEP", "scaled", "make_inputs", "bytes_per_elem",
