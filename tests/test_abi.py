@@ -2,6 +2,7 @@
 import ctypes as C
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -47,6 +48,30 @@ def test_binding_struct_layouts_match_header():
             for part in decl.split(","):
                 names.append(re.findall(r"\w+", part)[-1])
         assert names == [f[0] for f in cls._fields_], struct
+
+
+def test_binding_struct_offsets_match_the_compiled_header(tmp_path):
+    # byte offsets and sizes as a C compiler lays the header's structs out
+    fields = {"vattn_config": _abi.vattn_config, "vattn_params": _abi.vattn_params}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "vattn.h"', "int main(void) {"]
+    for struct, cls in fields.items():
+        lines.append(f'  printf("{struct} size %zu\\n", sizeof({struct}));')
+        for name, _ in cls._fields_:
+            lines.append(f'  printf("{struct} {name} %zu\\n", offsetof({struct}, {name}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
+                   check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        struct, name, val = line.split()
+        got[(struct, name)] = int(val)
+    for struct, cls in fields.items():
+        assert got[(struct, "size")] == C.sizeof(cls), struct
+        for name, _ in cls._fields_:
+            assert got[(struct, name)] == getattr(cls, name).offset, (struct, name)
 
 
 def test_strerror_without_device(lib):
