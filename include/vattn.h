@@ -54,7 +54,9 @@
  *   budgets    [batch][Hkv] int32: b (N_tail when the tail was taken whole,
  *              0 when there is no tail)
  *   head_need  [batch][Hq] int32: n_h, the CLT size required by query head
- *              hq (N_tail when the tail was taken whole before any pilot)
+ *              hq (N_tail when the tail was taken whole before any pilot); with
+ *              the output guarantee, the larger of the denominator's and the
+ *              numerator's sizes
  * A contiguous cache is one page per sequence: page_size >= max_ctx (a
  * multiple of 16) and page_table[b][0] = b.
  *
