@@ -46,7 +46,8 @@ def kernel_hash():
         parts[name] = text[pos:marks[i + 1][0] if i + 1 < len(marks) else len(text)]
     h = hashlib.sha256()
     for name in SCORE_SECTIONS:
-        h.update(parts[name].encode())
+        # a missing section changes the hash, so stale counters are not reported
+        h.update(parts.get(name, f"<no section {name}>").encode())
     return h.hexdigest()[:16]
 
 

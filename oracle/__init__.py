@@ -33,6 +33,7 @@ class Problem(C.Structure):
         ("pilot_min", C.c_int), ("pilot_num", C.c_int), ("pilot_den", C.c_int),
         ("eps", C.c_float), ("delta", C.c_float), ("seed", C.c_uint64),
         ("guarantee", C.c_int),
+        ("topp_num", C.c_int), ("topp_den", C.c_int),
     ]
 
 
@@ -141,7 +142,8 @@ def make_problem(w, seed=None, eps=None, batch=None, guarantee=None):
         pilot_min=w.pilot_min, pilot_num=w.pilot_num, pilot_den=w.pilot_den,
         eps=w.eps if eps is None else eps, delta=w.delta,
         seed=w.seed if seed is None else seed,
-        guarantee=GUARANTEES[guarantee or getattr(w, "guarantee", "denominator")])
+        guarantee=GUARANTEES[guarantee or getattr(w, "guarantee", "denominator")],
+        topp_num=getattr(w, "topp_num", 0), topp_den=getattr(w, "topp_den", 0))
 
 
 def decode(problem, inputs, units=None, L=None):

@@ -62,6 +62,7 @@ typedef struct {
   float eps, delta;
   uint64_t seed;
   int guarantee; /* ORC_GUARANTEE_DENOMINATOR or ORC_GUARANTEE_OUTPUT */
+  int topp_num, topp_den; /* topp_den > 0: top-p selection with p = topp_num / topp_den */
 } orc_problem;
 
 /* ------------------------------------------------------------------ */
@@ -284,7 +285,6 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
   const int wst = (N - pr->window) > s1 ? (N - pr->window) : s1;
   const int mlen = wst - s1;
   long long kb = pr->topk_den ? ((long long)N * pr->topk_num) / pr->topk_den : pr->topk_abs;
-  const int kk = (int)(kb < mlen ? kb : mlen);
   long long pb = pr->pilot_min;
   if (pr->pilot_den) {
     long long c = ((long long)N * pr->pilot_num + pr->pilot_den - 1) / pr->pilot_den;
@@ -342,16 +342,39 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
 
   /* Top-k over M: largest score first, equal scores to the lower position  */
   /* (reading: the pages give no tie rule). Key = ord(score) * 2^32 + (2^32-1-j). */
-  int32_t* topk = malloc(sizeof(int32_t) * (size_t)(kk > 0 ? kk : 1));
-  {
-    uint64_t* keys = malloc(sizeof(uint64_t) * (size_t)(mlen > 0 ? mlen : 1));
-    for (int j = s1; j < wst; j++)
-      keys[j - s1] = ((uint64_t)orc_ord(rs[j - s1]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
-    qsort(keys, (size_t)mlen, sizeof(uint64_t), cmp_u64_desc);
-    for (int i = 0; i < kk; i++) topk[i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(keys[i] & 0xFFFFFFFFu));
-    qsort(topk, (size_t)kk, sizeof(int32_t), cmp_i32_asc);
-    free(keys);
+  uint64_t* keys = malloc(sizeof(uint64_t) * (size_t)(mlen > 0 ? mlen : 1));
+  for (int j = s1; j < wst; j++)
+    keys[j - s1] = ((uint64_t)orc_ord(rs[j - s1]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+  qsort(keys, (size_t)mlen, sizeof(uint64_t), cmp_u64_desc);
+  int kk = (int)(kb < mlen ? kb : mlen);
+  if (pr->topp_den > 0) {
+    /* Top-p (reading: the pages name top-p selection as the mass-threshold   */
+    /* variant of top-k and give no formula): the smallest number of the     */
+    /* highest-ranked middle positions, in the key order above, whose share  */
+    /* of the middle's softmax mass under the scaled ranking scores reaches  */
+    /* p = topp_num / topp_den. Mass in 2^-32 fixed point, as the budget's:  */
+    /* x_j = vexp(fl(r_j c) - max_M fl(r c)), xq_j = rint(x_j 2^32), so the  */
+    /* cut is an exact integer comparison: prefix * den >= num * S.          */
+    float mx = -INFINITY;
+    for (int j = 0; j < mlen; j++) {
+      float sc = rs[j] * scale;
+      if (sc > mx) mx = sc;
+    }
+    uint64_t S = 0;
+    for (int j = 0; j < mlen; j++) S += (uint64_t)llrintf(orc_vexp(rs[j] * scale - mx) * 4294967296.0f);
+    const u128 target = (u128)S * (u128)(uint64_t)pr->topp_num;
+    u128 prefix = 0;
+    kk = 0;
+    while (kk < mlen && prefix * (u128)(uint64_t)pr->topp_den < target) {
+      const int j = (int)(0xFFFFFFFFu - (uint32_t)(keys[kk] & 0xFFFFFFFFu));
+      prefix += (u128)(uint64_t)llrintf(orc_vexp(rs[j - s1] * scale - mx) * 4294967296.0f);
+      kk++;
+    }
   }
+  int32_t* topk = malloc(sizeof(int32_t) * (size_t)(kk > 0 ? kk : 1));
+  for (int i = 0; i < kk; i++) topk[i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(keys[i] & 0xFFFFFFFFu));
+  qsort(topk, (size_t)kk, sizeof(int32_t), cmp_i32_asc);
+  free(keys);
 
   /* Deterministic set I_f, ascending; tail T = M minus top-k, ascending. */
   const int nI = s1 + kk + (N - wst);
@@ -570,6 +593,7 @@ int orc_decode(const orc_problem* pr, const void* q, const void* k_cache, const 
   if (!(pr->eps > 0.0f) || !(pr->delta > 0.0f && pr->delta < 1.0f)) return -1;
   if (pr->pilot_min < 2) return -1;
   if (pr->guarantee != ORC_GUARANTEE_DENOMINATOR && pr->guarantee != ORC_GUARANTEE_OUTPUT) return -1;
+  if (pr->topp_den < 0 || pr->topp_num < 0 || (pr->topp_den > 0 && pr->topp_num > pr->topp_den)) return -1;
   if (pr->sinks < 0 || pr->window < 0 || pr->topk_abs < 0 || pr->topk_num < 0 || pr->topk_den < 0 ||
       pr->pilot_num < 0 || pr->pilot_den < 0)
     return -1;

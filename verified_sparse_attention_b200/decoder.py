@@ -94,6 +94,8 @@ def decoder_for(w, device=None, max_batch=None):
 
 def params_for(w, inputs, eps=None, seed=None, guarantee=None):
     """vattn_params of a synthetic workload with its drawn inputs (device tensors)."""
+    if getattr(w, "topp_den", 0):
+        raise NotImplementedError("top-p selection is not built in the CUDA library")
     return SparseDecoder.make_params(
         sinks=w.sinks, window=w.window, topk_abs=w.topk_abs, topk_num=w.topk_num,
         topk_den=w.topk_den, pilot_min=w.pilot_min, pilot_num=w.pilot_num, pilot_den=w.pilot_den,

@@ -59,6 +59,8 @@ class Workload:
     data_seed: int
     recipe: str
     guarantee: str = "denominator"  # "denominator" | "output": what the budget bounds
+    topp_num: int = 0       # topp_den > 0: top-p selection, p = topp_num / topp_den
+    topp_den: int = 0       #   (the oracle only; the CUDA library selects a fixed k)
 
     @property
     def pages_per_seq(self):
@@ -217,7 +219,8 @@ def describe(w):
             f"N={'%d' % w.max_ctx if w.min_ctx == w.max_ctx else '%d..%d' % (w.min_ctx, w.max_ctx)} "
             f"ps{w.page_size} {w.proxy}{'' if w.proxy == 'exact' else ' r%d' % w.proxy_rank} "
             f"s{w.sinks} w{w.window} eps{w.eps} delta{w.delta}"
-            + ("" if w.guarantee == "denominator" else f" guarantee={w.guarantee}"))
+            + ("" if w.guarantee == "denominator" else f" guarantee={w.guarantee}")
+            + ("" if not w.topp_den else f" top-p {w.topp_num}/{w.topp_den}"))
 
 
 __all__ = ["Workload", "WORKLOADS", "PAGED_EPS_SWEEP", "scaled", "make_inputs", "bytes_per_elem",
