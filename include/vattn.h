@@ -22,8 +22,10 @@
  * exp(s_j - m)) by the same CLT condition (a reading; the pages give no
  * formula): n >= (z * N_tail / (eps * |Nv|))^2 * tr(Sigma), with tr(Sigma)
  * the sum over dimensions of the pilot's unbiased variance of x v, and |Nv|^2
- * the pilot's unbiased estimate (|Nv_hat|^2 - N_tail^2 tr(Sigma) / p; not
- * positive: the whole tail). Computed in double in a fixed order (items in
+ * replaced by a one-sided lower confidence bound from the pilot: with
+ * R = N_tail^2 tr(Sigma) / p the noise energy of the pilot mean and
+ * U = |Nv_hat|^2 - R, L = U - z sqrt(4 max(U, 0) R + 2 R^2) (not positive:
+ * the whole tail). Computed in double in a fixed order (items in
  * list order, then dimensions ascending), so it is reproducible bit for bit.
  * The ranking score is exact (q . k), a SparQ-style proxy over the r largest
  * query components ("SparQ Attention: Bandwidth-Efficient LLM Inference",

@@ -463,12 +463,12 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
         /* squared length is N_tail^2 tr(Sigma) / b, and                    */
         /*   n >= (z * N_tail / (eps * |Nv|))^2 * tr(Sigma),                */
         /* tr(Sigma) = sum over dims of the unbiased pilot variance of x v, */
-        /* |Nv| = length of (sum over I_f of x v) + N_tail * (pilot mean).  */
+        /* Nv_hat = (sum over I_f of x v) + N_tail * (pilot mean), and      */
+        /* |Nv|^2 its lower confidence bound below.                         */
         /* In double: each product x * v is exact (24 x 24 significant      */
         /* bits at most); sums run over I_f in list order and over the      */
         /* pilot in draw order, then over dims ascending. A negative        */
-        /* variance (rounding) counts as 0; |Nv| = 0 takes the whole tail   */
-        /* unless every variance is 0 as well.                              */
+        /* variance (rounding) counts as 0.                                 */
         double tr = 0.0, nsq = 0.0;
         for (int e = 0; e < d; e++) {
           double A = 0.0, T1 = 0.0, T2 = 0.0;
@@ -485,12 +485,23 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
           tr = tr + ve;
           nsq = nsq + Ne * Ne;
         }
-        /* the pilot mean's own noise adds N_tail^2 tr(Sigma) / p to |Nv|^2 */
-        /* in expectation; it is taken off (unbiased estimate of |Nv|^2)    */
-        double nsq_u = nsq - (((double)ntail * (double)ntail) / (double)p) * tr;
+        /* |Nv|^2 is sized from a one-sided lower confidence bound. The     */
+        /* pilot mean's noise, with covariance C = N_tail^2 Sigma / p and   */
+        /* energy R = tr(C), adds R to |Nv_hat|^2 in expectation, so         */
+        /* nsq_u = |Nv_hat|^2 - R is unbiased. Its variance is              */
+        /* 4 Nv' C Nv + 2 tr(C^2) <= 4 |Nv|^2 R + 2 R^2 (the largest         */
+        /* eigenvalue of C is at most its trace), so                        */
+        /*   L = nsq_u - z * sqrt(4 max(nsq_u, 0) R + 2 R^2)                */
+        /* undershoots |Nv|^2 with probability about delta / 2 or less.     */
+        /* When L is not positive the pilot cannot bound |Nv| away from 0   */
+        /* and the whole tail is taken (unless every variance is 0).        */
+        double R = (((double)ntail * (double)ntail) / (double)p) * tr;
+        double nsq_u = nsq - R;
+        double se2 = 4.0 * (nsq_u > 0.0 ? nsq_u : 0.0) * R + 2.0 * R * R;
+        double L = nsq_u - z * sqrt(se2);
         double need_v;
-        if (nsq_u > 0.0) {
-          double tv = (z * (double)ntail) / ((double)pr->eps * sqrt(nsq_u));
+        if (L > 0.0) {
+          double tv = (z * (double)ntail) / ((double)pr->eps * sqrt(L));
           need_v = (tv * tv) * tr;
         } else {
           need_v = tr > 0.0 ? (double)ntail : 0.0;

@@ -4,7 +4,8 @@ Same bar as the denominator-only parity tests: selected indices, counts,
 budgets and per-head sizes bit for bit (the numerator sizes are computed in
 double in a fixed order on both sides), outputs within 2e-3 (bf16) or 1e-5
 (fp32) per row. Coherent V (every element shifted by +1) keeps most budgets
-sampled; zero-mean V mostly takes every tail whole at small eps.
+sampled; zero-mean V mostly takes every tail whole, since a small pilot cannot
+bound |Nv| away from 0 there.
 """
 import numpy as np
 import pytest
@@ -38,6 +39,17 @@ def test_parity_reduced_coherent_v(name, eps):
 @pytest.mark.parametrize("name", ["tiny_f32", "gqa", "paged"])
 def test_parity_reduced_zero_mean_v(name):
     check(_out(SMALL[name], eps=0.5))
+
+
+def test_parity_sampled_numerator_budgets():
+    # the sampled branch of the lower confidence bound: a sharper query lets the
+    # planted keys carry |Nv|, so a 256-draw pilot samples zero-mean tails
+    w = _out(SMALL["tiny_f32"], eps=0.3, pilot_min=256)
+    x = synth.make_inputs(w)
+    x["q"] = x["q"] * 2.0
+    got, ref = check(w, inputs=x)
+    ntail = 4096 - 4 - 64 - 128
+    assert (got["budgets"] < ntail).any() and (got["budgets"] > 256).any(), got["budgets"]
 
 
 @pytest.mark.parametrize("G", [1, 2, 8])

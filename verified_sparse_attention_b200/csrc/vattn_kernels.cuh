@@ -2108,8 +2108,10 @@ __global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
 //   A = sum over I_f of x v_e;  T1, T2 = sums over the pilot of y, y * y, y = x v_e;
 //   var_e = max(0, (p T2 - T1^2) / (p (p - 1)));  Nv_e = A + N_tail T1 / p.
 // One thread per head then sums var_e and Nv_e^2 over e ascending into tr and
-// |Nv_hat|^2, takes off the pilot mean's own noise N_tail^2 tr / p, and writes
-//   n_v = (z N_tail / (eps |Nv|))^2 tr   (the whole tail when |Nv|^2 <= 0 < tr)
+// |Nv_hat|^2. The pilot mean's noise has energy R = N_tail^2 tr / p; the lower
+// confidence bound L = (|Nv_hat|^2 - R) - z sqrt(4 max(|Nv_hat|^2 - R, 0) R + 2 R^2)
+// stands for |Nv|^2, and the kernel writes
+//   n_v = (z N_tail / eps)^2 tr / L   (the whole tail when L <= 0 < tr)
 // to num_need; k_budget takes max(n_h, n_v). The items' row indices are
 // looked up once per block of kNumOffItems items (one parallel pass over
 // sel and the page table); the V rows and the true scores of each round of
@@ -2236,10 +2238,15 @@ __global__ void __launch_bounds__(kNumThreads) k_numstats(DevParams P) {
       tr = __dadd_rn(tr, s_red[0][tid * D + k]);
       nsq = __dadd_rn(nsq, s_red[1][tid * D + k]);
     }
-    const double nsq_u = __dsub_rn(nsq, __dmul_rn(__ddiv_rn(__dmul_rn(nt, nt), pd), tr));
+    // lower confidence bound of |Nv|^2: nsq_u - z * sqrt(4 max(nsq_u, 0) R + 2 R^2)
+    const double R = __dmul_rn(__ddiv_rn(__dmul_rn(nt, nt), pd), tr);
+    const double nsq_u = __dsub_rn(nsq, R);
+    const double se2 = __dadd_rn(__dmul_rn(__dmul_rn(4.0, nsq_u > 0.0 ? nsq_u : 0.0), R),
+                                 __dmul_rn(__dmul_rn(2.0, R), R));
+    const double lcb = __dsub_rn(nsq_u, __dmul_rn(P.z, __dsqrt_rn(se2)));
     double need;
-    if (nsq_u > 0.0) {
-      const double tv = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), __dsqrt_rn(nsq_u)));
+    if (lcb > 0.0) {
+      const double tv = __ddiv_rn(__dmul_rn(P.z, nt), __dmul_rn(static_cast<double>(P.eps), __dsqrt_rn(lcb)));
       need = __dmul_rn(__dmul_rn(tv, tv), tr);
     } else {
       need = tr > 0.0 ? nt : 0.0;
