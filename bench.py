@@ -8,6 +8,10 @@ One step = one vattn_decode call over the whole batch of the workload (every
 row of the hot path: query prep, ranking-score pass, top-k select, pilot,
 budget, gather, combine). Inputs are resident in HBM before the timed region
 and larger than L2 (so no flush is needed). Prints one JSON line (rank 0).
+The headline is --workload (default gqa_32k); at one GPU the line also carries
+`per_config`, the same measurements for the other long-context workloads
+(sparq_128k, loki_64k, paged_sweep at eps 0.05). The score pass's roofline is
+timed by events on SCORE_SAMPLES further calls after the timed region.
 Under torchrun each rank runs its own batch on its own GPU (weak scaling; no
 collective on the data path, one max-reduction of the elapsed time).
 """
@@ -30,6 +34,10 @@ from verified_sparse_attention_b200 import _abi, ranks, synth  # noqa: E402
 from verified_sparse_attention_b200.decoder import decoder_for, params_for  # noqa: E402
 
 METRIC = "sparse decode-attn calls/s & achieved HBM GB/s (% of ~8 TB/s) at 32k–128k ctx"
+NOMINAL_HBM_GBS = 8000.0
+SCORE_SAMPLES = 64   # score passes timed by events after the timed region
+# the other long-context workloads measured in the same run (name, eps override)
+PER_CONFIG = [("sparq_128k", None), ("loki_64k", None), ("paged_sweep", 0.05)]
 KERNEL_SOURCE = "verified_sparse_attention_b200/csrc/vattn_kernels.cuh"
 # the sections of KERNEL_SOURCE that hold the ranking-score pass (its kernels
 # and their own helpers): the DRAM counters in profiles/ are keyed to them
@@ -80,8 +88,12 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, index, period=0.005):
+        """index None: sample nothing."""
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.ok = period, False
+        self._stop = threading.Event()
+        if index is None:
+            return
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -91,7 +103,6 @@ class ClockSampler:
             self.ok = True
         except Exception:
             self.ok = False
-        self._stop = threading.Event()
 
     def _run(self):
         while not self._stop.is_set():
@@ -132,7 +143,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ byte accounting
 def algorithmic_bytes(w, x, res):
-    """(score-pass bytes per launch, whole-call KV bytes) from the call's own outputs."""
+    """Bytes one call must move, from the call's own outputs: the score pass's K (or
+    proxy) rows of the middle, the 4-byte ranking keys it writes (workspace, reported
+    apart), and the gathers' K and V rows of every selected entry."""
     e = synth.bytes_per_elem(w)
     d = w.head_dim
     n = x["seq_lens"].to(torch.int64).cpu()
@@ -140,7 +153,7 @@ def algorithmic_bytes(w, x, res):
     wst = torch.maximum(n - w.window, s1)
     mid = (wst - s1).clamp(min=0)                          # middle rows per sequence
     per_row = {"exact": d * e, "sparq": w.proxy_rank * e, "loki": w.proxy_rank * e}[w.proxy]
-    score = int(mid.sum()) * w.num_kv_heads * (per_row + 4)     # K (or proxy) read + key write
+    rows = int(mid.sum()) * w.num_kv_heads
     cnt = res["sel_count"].to(torch.int64).cpu()            # [B, Hkv] rows gathered (K and V)
     gather = int(cnt.sum()) * 2 * d * e
     if w.guarantee == "output":
@@ -153,18 +166,18 @@ def algorithmic_bytes(w, x, res):
         n_if = s1 + k + (n - wst)
         piloted = (mid - k) > p
         gather += int(((n_if + p) * piloted).sum()) * w.num_kv_heads * d * e
-    return score, score + gather
+    return {"score_read": rows * per_row, "key_write": rows * 4, "gather": gather,
+            "call": rows * per_row + gather}
 
 
-# ------------------------------------------------------------------ arms
-def run_gpu_arm(args, rank, world, local_rank):
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[args.workload].replace(guarantee=args.guarantee)
-    w = ranks.rank_workload(w, rank)
+# ------------------------------------------------------------------ one workload
+def run_config(w, args, dev, world, steps, *, headline):
+    """Time `steps` decode calls of workload w (inputs resident in HBM, larger than L2),
+    then 64 more with the score pass timed by events, then the dense decode on the same
+    inputs. Returns (decoder, inputs, result dict)."""
     x = synth.make_inputs(w, device=dev)
     dec = decoder_for(w, device=dev)
-    prm = params_for(w, x, eps=args.eps)
+    prm = params_for(w, x)
     outs = dec.alloc_outputs(w.batch)
     stream = torch.cuda.current_stream()
 
@@ -183,65 +196,88 @@ def run_gpu_arm(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     if dec.last_error():
-        raise RuntimeError("device error word set during warm-up")
+        raise RuntimeError(f"{w.name}: device error word set during warm-up")
     launches_per_call = _abi.vattn_last_launch_count(dec.ctx)
-    _abi.vattn_score_pass_ms(dec.ctx, reset=True)
-    # the score pass of one call in 16 is timed by events on the launching
-    # stream (an event pair stops that call's kernel from overlapping its
-    # neighbours, so the other calls run undisturbed)
-    _abi.vattn_set_timing(dec.ctx, 16)
 
     ranks.barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with (ClockSampler(torch.cuda.current_device()) if headline else ClockSampler(None)) as clk:
         t0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         t1.record(stream)
         torch.cuda.synchronize()
     ranks.barrier(world)
-    _abi.vattn_set_timing(dec.ctx, False)
     ms = t0.elapsed_time(t1)
-    score_ms, score_n = _abi.vattn_score_pass_ms(dec.ctx, reset=True)
     ms_max = ranks.max_over_ranks(ms, world, dev)
 
-    score_bytes, call_bytes = algorithmic_bytes(w, x, outs)
+    # the score pass alone: an event pair on the launching stream around it in each of
+    # SCORE_SAMPLES further calls (the pair stops it overlapping its neighbours, so
+    # these calls are kept out of the timed region above)
+    _abi.vattn_score_pass_ms(dec.ctx, reset=True)
+    _abi.vattn_set_timing(dec.ctx, 1)
+    for _ in range(SCORE_SAMPLES):
+        step()
+    torch.cuda.synchronize()
+    _abi.vattn_set_timing(dec.ctx, 0)
+    score_ms, score_n = _abi.vattn_score_pass_ms(dec.ctx, reset=True)
+    if dec.last_error():
+        raise RuntimeError(f"{w.name}: device error word set")
+
+    nbytes = algorithmic_bytes(w, x, outs)
     budgets = outs["budgets"].cpu()
 
     # dense decode attention on the same inputs (comparison baseline)
+    dsteps = max(10, min(steps, 200))
     for _ in range(args.warmup):
         dec.dense(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"],
                   x["num_pages"], stream=stream)
     torch.cuda.synchronize()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     d0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(dsteps):
         dec.dense(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"],
                   x["num_pages"], stream=stream)
     d1.record(stream)
     torch.cuda.synchronize()
-    dense_ms = d0.elapsed_time(d1) / args.steps
+    dense_ms = d0.elapsed_time(d1) / dsteps
 
-    e2e = run_e2e(args, w, x, dec, prm, stream, dev, world)
+    return dec, x, prm, dict(w=w, ms=ms_max, steps=steps, score_ms=score_ms, score_n=score_n,
+                             bytes=nbytes, budgets=budgets, launches_per_call=launches_per_call,
+                             clocks=clk.summary() if headline else None, dense_ms=dense_ms)
 
-    result = dict(w=w, x=x, ms=ms_max, score_ms=score_ms, score_n=score_n,
-                  score_bytes=score_bytes, call_bytes=call_bytes, budgets=budgets,
-                  launches=launches_per_call * args.steps, clocks=clk.summary(),
-                  dense_ms=dense_ms, e2e=e2e)
-    return dec, result
+
+def summarize(r, world, peak):
+    """Rates of one run_config result: calls/s, the score pass's roofline, whole-call GB/s."""
+    calls_s = ranks.job_rate(world, r["steps"], r["ms"])
+    call_s = r["ms"] / 1e3 / r["steps"]
+    avg_score_s = (r["score_ms"] / max(1, r["score_n"])) / 1e3
+    b = r["bytes"]
+    achieved = b["score_read"] / avg_score_s / 1e9
+    return {"calls_per_s": calls_s, "us_per_call": call_s * 1e6,
+            "score_pass": {"achieved_gbs": achieved, "frac": achieved / peak,
+                           "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                           "avg_launch_us": avg_score_s * 1e6, "samples": r["score_n"],
+                           "read_bytes_per_launch": b["score_read"],
+                           "key_write_bytes_per_launch": b["key_write"]},
+            "call_kv_bytes": b["call"], "call_achieved_gbs": b["call"] / call_s / 1e9,
+            "call_frac_of_peak": b["call"] / call_s / 1e9 / peak,
+            "dense_calls_per_s": world / (r["dense_ms"] / 1e3),
+            "speedup_vs_dense": r["dense_ms"] / (r["ms"] / r["steps"]),
+            "budget_mean": float(r["budgets"].float().mean())}
 
 
 def run_e2e(args, w, x, dec, prm, stream, dev, world):
     """Same metric through the C ABI with host buffers: pinned host -> device copies of
-    every input and a device -> host read of the result inside the timed region."""
+    every input and a device -> host read of every result (out, sel_idx, sel_count,
+    budgets, head_need) inside the timed region."""
     keys = ["q", "k_cache", "v_cache", "page_table", "seq_lens"]
     extra = [k for k in ("k_t_cache", "k_proj_cache", "proj_basis") if k in x]
     host = {k: x[k].cpu().pin_memory() for k in keys + extra}
     devb = {k: torch.empty_like(x[k]) for k in keys + extra}
     outs = dec.alloc_outputs(w.batch)
-    out_h = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-             for k, v in outs.items() if k != "sel_idx"}
+    out_h = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
     p = params_for(w, {**devb, "num_pages": x["num_pages"]}, eps=args.eps)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(v.numel() * v.element_size() for v in out_h.values())
@@ -333,6 +369,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the other long-context workloads")
+    ap.add_argument("--per-config-steps", type=int, default=200)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -374,40 +413,68 @@ def main():
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dec, r = run_gpu_arm(args, rank, world, local_rank)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
     peak, peak_kind = load_peaks()
-    w = r["w"]
-    calls_s = ranks.job_rate(world, args.steps, r["ms"])
-    avg_score_s = (r["score_ms"] / max(1, r["score_n"])) / 1e3
-    achieved = r["score_bytes"] / avg_score_s / 1e9
-    call_s = r["ms"] / 1e3 / args.steps
-    line = {"metric": METRIC, "value": calls_s, "unit": "calls/s", "n_gpus": world,
+    wr = ranks.rank_workload(w, rank)
+    dec, x, prm, r = run_config(wr, args, dev, world, args.steps, headline=True)
+    sm = summarize(r, world, peak)
+    sp = sm["score_pass"]
+    e2e = run_e2e(args, wr, x, dec, prm, torch.cuda.current_stream(), dev, world)
+    line = {"metric": METRIC, "value": sm["calls_per_s"], "unit": "calls/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic", "config": cfg,
-            "roofline": {"bound": "hbm", "kernel": "score pass (k_score_tma / k_score_rows / k_score_sparq)",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak,
+            "roofline": {"bound": "hbm",
+                         "kernel": "score pass (k_score_tma / k_score_rows / k_score_sparq)",
+                         "achieved": sp["achieved_gbs"], "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": sp["frac"],
+                         "frac_of_nominal_8tbs": sp["frac_of_nominal_8tbs"],
                          "traffic": profiled_traffic(w.name),
-                         "algorithmic_bytes_per_launch": r["score_bytes"],
-                         "avg_launch_us": avg_score_s * 1e6},
-            "call_kv_bytes": r["call_bytes"],
-            "call_achieved_gbs": r["call_bytes"] / call_s / 1e9,
-            "call_frac_of_peak": r["call_bytes"] / call_s / 1e9 / peak,
-            "dense_calls_per_s": world / (r["dense_ms"] / 1e3),
-            "budget_mean": float(r["budgets"].float().mean()),
-            "gpu_launches": r["launches"], "clocks": r["clocks"], "e2e": r["e2e"]}
+                         "algorithmic_bytes_per_launch": sp["read_bytes_per_launch"],
+                         "key_write_bytes_per_launch": sp["key_write_bytes_per_launch"],
+                         "avg_launch_us": sp["avg_launch_us"], "samples": sp["samples"]},
+            "call_kv_bytes": sm["call_kv_bytes"], "call_achieved_gbs": sm["call_achieved_gbs"],
+            "call_frac_of_peak": sm["call_frac_of_peak"],
+            "dense_calls_per_s": sm["dense_calls_per_s"],
+            "speedup_vs_dense": sm["speedup_vs_dense"], "budget_mean": sm["budget_mean"],
+            "gpu_launches": r["launches_per_call"] * args.steps, "clocks": r["clocks"],
+            "e2e": e2e}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in r["x"].items()}
-        val, done, el = time_oracle(w, cpu, args.cpu_budget_s)
+        cpu = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in x.items()}
+        val, done, el = time_oracle(wr, cpu, args.cpu_budget_s)
         line["cpu_baseline"] = {"value": val, "unit": "calls/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} (sequence, KV head) units of a {w.units}-unit call "
                                           f"in {el:.1f}s, single-threaded C oracle"}
-        val, done, el, T = time_oracle_all_cores(w, cpu, args.cpu_budget_s)
+        val, done, el, T = time_oracle_all_cores(wr, cpu, args.cpu_budget_s)
         line["cpu_baseline_all_cores"] = {
             "value": val, "unit": "calls/s", "cores": T, "kind": "oracle",
             "sample": f"{done} units in {el:.1f}s, one unit per call on {T} threads of the same C oracle"}
+        del cpu
     dec.close()
+    del x, dec
+    torch.cuda.empty_cache()
+
+    # the other long-context workloads, same rules, at one GPU only (their inputs are
+    # made after the headline's are freed)
+    if world == 1 and args.per_config and args.guarantee == "denominator":
+        per = {}
+        for name, eps in PER_CONFIG:
+            if name == w.name:
+                continue
+            wc = synth.WORKLOADS[name]
+            if eps is not None:
+                wc = wc.replace(eps=eps)
+            dec_c, x_c, _, rc = run_config(wc, args, dev, world, max(args.steps, args.per_config_steps),
+                                           headline=False)
+            smc = summarize(rc, world, peak)
+            smc["score_pass"]["traffic"] = profiled_traffic(name)
+            smc["workload"] = synth.describe(wc)
+            per[name] = smc
+            dec_c.close()
+            del x_c, dec_c
+            torch.cuda.empty_cache()
+        line["per_config"] = per
     if ranks.reports(rank):
         emit(line)
     if world > 1:

@@ -165,9 +165,12 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
 
    Scratch: a fixed array of 8 MiB per device, defined in the library. A call
    needs batch * Hq * (head_dim + 2) * 4 bytes of it at least; a larger call
-   returns VATTN_ESCRATCH before touching the device. The first call made with
-   a device current looks up that device's copy of the array (and its SM
-   count); make that first call before any stream capture begins. Every later
+   returns VATTN_ESCRATCH before touching the device. The first call made
+   under a CUDA context looks up that device's copy of the array (and its SM
+   count); a call under a different context on the same device (after
+   cudaDeviceReset, or with a driver-API context current) looks it up again,
+   since the old address belongs to the old context. Make the first call of
+   each context before any stream capture begins. Every later
    call on the device shares the same array: it keeps the last call's partial
    results, nothing in it needs to start at zero (a call writes every part it
    reads), and calls that overlap in time on one device race and corrupt
@@ -183,6 +186,17 @@ int vattn_dense_decode_static(const vattn_config* cfg, const void* q, const void
    word (VATTN_DEV_* bits). sync == 0: return the host status of the last
    call on this context, without touching the device. */
 int vattn_last_error(vattn_ctx* ctx, int sync);
+
+/* Self-check of the device error path: launches one warp on `stream` that
+   waits, with a limit of `tries` tries (1 .. 2^20), on a barrier that no copy
+   ever completes, exactly as the kernels' copy rings wait for their copies,
+   and sets VATTN_DEV_TIMEOUT in the context's error word when the limit runs
+   out (it always does). The kernel then returns normally; nothing is left in
+   flight, and the context stays usable. vattn_last_error(ctx, 1) reports and
+   clears the bit. Returns VATTN_EINVAL for a bad argument. (No counterpart in
+   the pages: it exists so that the timeout path can be tested without a
+   fault.) */
+int vattn_check_bounded_wait(vattn_ctx* ctx, int tries, void* stream);
 
 /* Bytes of device workspace the context holds. */
 size_t vattn_workspace_bytes(const vattn_ctx* ctx);

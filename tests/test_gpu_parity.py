@@ -213,6 +213,25 @@ def test_bad_length_sets_error():
     assert np.all(got["out"] == 0)
 
 
+def test_bounded_wait_runs_out_and_reports_a_timeout():
+    # a wait on a barrier that no copy completes: the kernel gives up after its
+    # limit, sets VATTN_DEV_TIMEOUT and returns; the context stays usable
+    w = SMALL["tiny_f32"]
+    dev = _cuda()
+    dec = decoder_for(w)
+    try:
+        assert dec.last_error() == 0
+        for tries in (1, 1000):
+            _abi.vattn_check_bounded_wait(dec.ctx, tries)
+            assert dec.last_error() == _abi.VATTN_DEV_TIMEOUT  # read and cleared
+            assert dec.last_error() == 0
+        assert _abi.vattn_check_bounded_wait(dec.ctx, 0, check=False) == _abi.VATTN_EINVAL
+        assert _abi.vattn_check_bounded_wait(dec.ctx, (1 << 20) + 1, check=False) == _abi.VATTN_EINVAL
+    finally:
+        dec.close()
+    check(w)  # a decode on the same device afterwards is still exact
+
+
 def test_host_argument_checks():
     w = SMALL["tiny_f32"]
     dev = _cuda()

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from tests.helpers import rel_err_rows
+from tests.helpers import dense_attention, rel_err_rows
 from verified_sparse_attention_b200 import _abi, synth
 
 TOL = {"bf16": 2e-3, "f32": 1e-5}
@@ -84,3 +84,44 @@ def test_two_calls_in_a_row_match_the_context_entry(first, second):
         assert np.isfinite(got).all()
         err = rel_err_rows(got.reshape(-1, w.head_dim), ref.reshape(-1, w.head_dim))
         assert err.max() <= TOL[w.dtype], (w.name, float(err.max()))
+        # and against float64 dense attention computed from the caches
+        for b in range(w.batch):
+            for hq in range(0, w.num_q_heads, max(1, w.num_q_heads // 4)):
+                e = rel_err_rows(got[b, hq], dense_attention(cpu, w, b, hq))
+                assert e <= TOL[w.dtype], (w.name, b, hq, float(e))
+
+
+@pytest.mark.gpu
+def test_bad_sequences_give_zero_rows_and_leave_the_others_alone():
+    # a page id past the pool, a length above max_ctx and an empty sequence: their
+    # rows are exactly 0 (there is no error word without a context); the other
+    # sequences match the context entry point on the same inputs
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = synth.scaled(synth.WORKLOADS["paged_sweep"], max_ctx=3000, min_ctx=1500, batch=5,
+                     data_seed=15)
+    cpu = synth.make_inputs(w)
+    cpu["page_table"][1, 7] = cpu["num_pages"] + 3
+    cpu["seq_lens"][2] = w.max_ctx + 1
+    cpu["seq_lens"][3] = 0
+    x = {k: (v.to("cuda") if hasattr(v, "to") else v) for k, v in cpu.items()}
+    for _ in range(2):  # the second call finds the first one's records in the array
+        got = _dense_static(w, x)
+        assert np.all(got[1:4] == 0.0)
+        ref = _dense_with_context_any_error(w, x)
+        for b in (0, 4):
+            err = rel_err_rows(got[b], ref[b])
+            assert err.max() <= TOL[w.dtype], (b, float(err.max()))
+
+
+def _dense_with_context_any_error(w, x):
+    ctx = _abi.vattn_create(_config(w))
+    try:
+        out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=torch.float32, device="cuda")
+        _abi.vattn_dense_decode(ctx, x["q"], x["k_cache"], x["v_cache"], x["page_table"],
+                                x["seq_lens"], w.batch, x["num_pages"], out)
+        torch.cuda.synchronize()
+        assert _abi.vattn_last_error(ctx) != 0  # the context entry point reports the bad rows
+        return out.cpu().numpy()
+    finally:
+        _abi.vattn_destroy(ctx)

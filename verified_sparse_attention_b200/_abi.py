@@ -19,7 +19,7 @@ VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE, VATTN_DEV_TIMEOUT = 1, 2, 4
 
 # every symbol include/vattn.h declares
 EXPORTS = ("vattn_create", "vattn_decode", "vattn_dense_decode", "vattn_dense_decode_static",
-           "vattn_last_error",
+           "vattn_last_error", "vattn_check_bounded_wait",
            "vattn_workspace_bytes", "vattn_set_timing", "vattn_score_pass_ms",
            "vattn_last_launch_count", "vattn_strerror", "vattn_destroy")
 
@@ -64,6 +64,8 @@ def lib():
         L.vattn_dense_decode.restype = I
         L.vattn_dense_decode_static.argtypes = [C.POINTER(vattn_config), P, P, P, P, P, I, I, P, P]
         L.vattn_dense_decode_static.restype = I
+        L.vattn_check_bounded_wait.argtypes = [P, I, P]
+        L.vattn_check_bounded_wait.restype = I
         L.vattn_last_error.argtypes = [P, I]
         L.vattn_last_error.restype = I
         L.vattn_workspace_bytes.argtypes = [P]
@@ -145,6 +147,12 @@ def vattn_dense_decode_static(config, q, k_cache, v_cache, page_table, seq_lens,
 
 def vattn_last_error(ctx, sync=True):
     return lib().vattn_last_error(ctx, 1 if sync else 0)
+
+
+def vattn_check_bounded_wait(ctx, tries, stream=None, check=True):
+    """Run the device wait self-check (sets VATTN_DEV_TIMEOUT in the error word)."""
+    rc = lib().vattn_check_bounded_wait(ctx, int(tries), _stream_ptr(stream))
+    return _check(rc, "vattn_check_bounded_wait") if check else rc
 
 
 def vattn_workspace_bytes(ctx):

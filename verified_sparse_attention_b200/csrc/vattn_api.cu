@@ -450,6 +450,12 @@ int vattn_last_error(vattn_ctx* ctx, int sync) {
   return static_cast<int>(v);
 }
 
+int vattn_check_bounded_wait(vattn_ctx* ctx, int tries, void* stream) {
+  if (!ctx || tries < 1 || tries > vattn::kWaitTries) return VATTN_EINVAL;
+  vattn::k_wait_check<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctx->err, tries);
+  return cudaGetLastError() == cudaSuccess ? VATTN_OK : VATTN_ECUDA;
+}
+
 int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void* v_cache,
                  const int32_t* page_table, const int32_t* seq_lens, int batch,
                  const vattn_params* prm, float* out, int32_t* sel_idx, int32_t* sel_count,

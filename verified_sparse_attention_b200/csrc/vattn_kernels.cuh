@@ -886,10 +886,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned by
                : "memory");
 }
 // Bounded wait for the completion of the barrier phase with parity `parity`;
-// false when the limit ran out (each try may itself suspend for a while).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+// false when `tries` tries ran out (each try may itself suspend for a while,
+// so the default limit ends a wait that can never complete in about a second).
+// A kernel whose wait failed issues no further copies into the ring; copies it
+// had issued before may still be landing in its shared memory when it exits,
+// the one hazard left after a timeout (it can only follow a copy that never
+// completes, which the row bounds of every copy rule out in normal operation).
+constexpr int kWaitTries = 1 << 20;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, int tries = kWaitTries) {
   const unsigned a = smem_u32(bar);
-  for (int it = 0; it < (1 << 20); it++) {
+  for (int it = 0; it < tries; it++) {
     unsigned done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
@@ -2264,6 +2270,23 @@ __global__ void __launch_bounds__(kCombGroups * D) k_combine(DevParams P) {
   grid_dependency_wait();
   unit_combine<D, G, MODE>(P, blockIdx.x, blockIdx.y);
   grid_dependents_launch();
+}
+
+// ============================================================ k_wait_check
+// Exercises the bounded-wait error path: one warp arms an mbarrier for 16
+// bytes that no copy ever delivers (no copy is issued, so nothing is in
+// flight at exit), waits with a limit of `tries`, and on timeout sets
+// VATTN_DEV_TIMEOUT in the error word, exactly as the copy rings do.
+__global__ void __launch_bounds__(32) k_wait_check(unsigned* err, int tries) {
+  __shared__ __align__(8) uint64_t s_bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_arrive_expect_tx(&s_bar, 16u);
+  __syncwarp();
+  if (!__all_sync(0xffffffffu, mbar_wait(&s_bar, 0u, tries)) && threadIdx.x == 0) atomicOr(err, kDevTimeout);
 }
 
 }  // namespace vattn

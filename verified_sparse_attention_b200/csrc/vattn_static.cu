@@ -3,7 +3,8 @@
 // The other entry points keep their scratch in a context workspace that
 // vattn_create allocates. This one needs no context: its only scratch is the
 // file-scope device array below, of a fixed size, whose address is looked up
-// once per device. It exists for callers that cannot allocate device memory
+// once per CUDA context (normally once per device; again after a device
+// reset). It exists for callers that cannot allocate device memory
 // at the point of the call (a server that has handed all free memory to its
 // KV-cache pool, code that must not risk the device-wide synchronisation a
 // free can cause, or a plug-in that cannot keep a context between calls).
@@ -19,6 +20,7 @@
 // in the array has to start at zero and the previous call's contents are
 // harmless. Two calls that overlap in time on one device (other streams,
 // other host threads) share the array and race: order them.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -276,31 +278,67 @@ bool pick(const vattn_config& c, int G, SplitFn* s, MergeFn* m) {
   return c.head_dim == 128 ? pick_g<float, 128>(G, s, m) : pick_g<float, 64>(G, s, m);
 }
 
-// Per-device set-up, done by the first call made with that device current:
-// the address of this device's copy of the array, and its SM count.
+// Per-context set-up: the address of this device's copy of the array, and
+// its SM count, looked up by the first call made with a given CUDA context
+// current on the device. The address belongs to the context that loaded the
+// module, so the slot remembers that context's id and the look-up is redone
+// when another context becomes current on the device (after
+// cudaDeviceReset, or a context made by the driver API), instead of handing
+// a kernel a stale address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
 struct DeviceSlot {
   bool ready;
+  unsigned long long ctx_id;
   float* scratch;
   int num_sms;
 };
 std::mutex g_slots_mu;
 DeviceSlot g_slots[kMaxDevices];
 
+template <typename Fn>
+Fn driver_entry(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Id of the context current on this thread (0 when none is current yet).
+int current_ctx_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return VATTN_ECUDA;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS) return VATTN_ECUDA;
+  *id = 0;
+  if (c && get_id(c, id) != CUDA_SUCCESS) return VATTN_ECUDA;
+  return VATTN_OK;
+}
+
 int device_slot(DeviceSlot* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return VATTN_ECUDA;
   if (dev < 0 || dev >= kMaxDevices) return VATTN_EINVAL;
+  unsigned long long id = 0;
+  if (const int rc = current_ctx_id(&id)) return rc;
   std::lock_guard<std::mutex> lock(g_slots_mu);
   DeviceSlot& s = g_slots[dev];
-  if (!s.ready) {
+  if (!s.ready || id == 0 || s.ctx_id != id) {
+    // the look-up also makes the runtime's primary context current if none was
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dense_scratch) != cudaSuccess || p == nullptr) return VATTN_ECUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
       return VATTN_ECUDA;
+    if (id == 0 && current_ctx_id(&id) != VATTN_OK) return VATTN_ECUDA;
     s.scratch = static_cast<float*>(p);
     s.num_sms = sms;
-    s.ready = true;
+    s.ctx_id = id;
+    s.ready = id != 0;
   }
   *out = s;
   return VATTN_OK;
