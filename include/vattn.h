@@ -135,6 +135,17 @@ typedef struct {
   int guarantee;     /* VATTN_GUARANTEE_DENOMINATOR (0) or VATTN_GUARANTEE_OUTPUT;  */
                      /* OUTPUT adds one kernel that reads the V rows of I_f and the */
                      /* pilot once more; anything else: VATTN_EINVAL                */
+  /* Top-p selection (the pages name top-k "(or top-p)" selection as the
+     predictor of the deterministic set; "vAttention: A New Approach to Sparse
+     Attention with Guaranteed Accuracy", third paragraph). topp_den > 0
+     replaces the fixed top-k (topk_* are then ignored): the predicted set is
+     the smallest number of the highest-ranked middle positions (ranking order,
+     ties to the lower position) whose share of the middle's softmax mass under
+     the scaled ranking scores reaches p = topp_num / topp_den, the mass taken
+     in 2^-32 fixed point (w_j = rint(exp(r_j/sqrt(d) - max) * 2^32), exp the
+     budget's fixed-order exp) so that the cut is the exact integer test
+     prefix * den >= num * S. 0 <= topp_num <= topp_den; topp_den = 0: off. */
+  int topp_num, topp_den;
 } vattn_params;
 
 /* Create a context on the current CUDA device and allocate its workspace.

@@ -139,7 +139,8 @@ def test_invalid_p_is_rejected(num, den):
         _decode(TINY.replace(topp_num=num, topp_den=den), synth.make_inputs(TINY))
 
 
-def test_the_cuda_binding_refuses_top_p():
-    w = TINY.replace(topp_num=1, topp_den=2)
-    with pytest.raises(NotImplementedError):
-        params_for(w, {"num_pages": 1})
+def test_the_binding_passes_p_through():
+    w = TINY.replace(topp_num=9, topp_den=10)
+    prm = params_for(w, {"num_pages": 1})
+    assert (prm.topp_num, prm.topp_den) == (9, 10)
+    assert params_for(TINY, {"num_pages": 1}).topp_den == 0

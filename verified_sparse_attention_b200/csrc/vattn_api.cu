@@ -479,6 +479,7 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   if (prm->num_pages < 1) return VATTN_EINVAL;
   if (prm->guarantee != VATTN_GUARANTEE_DENOMINATOR && prm->guarantee != VATTN_GUARANTEE_OUTPUT)
     return VATTN_EINVAL;
+  if (prm->topp_den < 0 || prm->topp_num < 0 || prm->topp_num > prm->topp_den) return VATTN_EINVAL;
   if (c.proxy == VATTN_SPARQ && (!prm->k_t_cache || !aligned16(prm->k_t_cache))) return VATTN_EINVAL;
   if (c.proxy == VATTN_LOKI && (!prm->k_proj_cache || !prm->proj_basis || !aligned16(prm->k_proj_cache)))
     return VATTN_EINVAL;
@@ -509,6 +510,8 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.seed = prm->seed;
   P.num_pages = prm->num_pages;
   P.guarantee = prm->guarantee == VATTN_GUARANTEE_OUTPUT;
+  P.topp_num = prm->topp_num;
+  P.topp_den = prm->topp_den;
   if (const int rc = encode_row_maps(c, k_cache, v_cache, prm->num_pages, &P)) return ctx->last_status = rc;
   P.q = q;
   P.k = k_cache;
@@ -550,6 +553,8 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
     cudaEventRecord(ctx->ev_stop[ctx->ev_used], st);
     ctx->ev_used++;
   }
+  // top-p: each unit's top-k size from the mass of its ranking scores
+  if (P.topp_den > 0) launch(vattn::k_topp, dim3(P.units), dim3(vattn::kToppThreads), 0, st, P, &launches);
   if (ctx->select1) {
     launch(vattn::k_select1, dim3(P.units), dim3(vattn::kSel1Threads), vattn::kSel1Smem, st, P, &launches);
   } else {

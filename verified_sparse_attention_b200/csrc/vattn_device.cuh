@@ -63,6 +63,7 @@ struct DevParams {
   unsigned long long seed;
   int nseg, dense;
   int guarantee;    // 1: the budget also bounds the numerator vector (output guarantee)
+  int topp_num, topp_den;  // topp_den > 0: top-p selection with p = topp_num / topp_den
   int CD, CS;       // grid sizes of the det (and dense) and sample gathers
   // inputs
   const void* q;
@@ -91,7 +92,7 @@ struct DevParams {
   int* num_need;    // [units][G]: numerator sizes n_v (output guarantee)
   int hist_words;   // histogram words per unit that k_prep zeroes (all only for the grid-wide select)
   long long* prefix;// [units + 1]: score-pass work prefix
-  unsigned* gcnt;   // [0]: score-pass chunks handed out (zeroed by k_prep)
+  unsigned* gcnt;   // [0]: score-pass chunks handed out, [1]: units done by k_topp (zeroed by k_prep)
   long long* pre_det;   // [2 units + 1]: slice prefix of the det (or dense) gather
   long long* pre_samp;  // [2 units + 1]: slice prefix of the sample gather
   float* rec_det;   // [CD + 2 units][G][2 + D]: det (or dense) gather records

@@ -52,8 +52,10 @@ __device__ __forceinline__ Regions regions(const DevParams& P, int n) {
   r.s1 = min(P.sinks, n);
   r.wst = max(n - P.window, r.s1);
   const int mlen = r.wst - r.s1;
-  const long long kb = P.topk_den ? (static_cast<long long>(n) * P.topk_num) / P.topk_den
-                                  : static_cast<long long>(P.topk_abs);
+  // with top-p the size is found after the score pass (k_topp); 0 until then
+  const long long kb = P.topp_den ? 0LL
+                       : P.topk_den ? (static_cast<long long>(n) * P.topk_num) / P.topk_den
+                                    : static_cast<long long>(P.topk_abs);
   r.k = static_cast<int>(min(kb, static_cast<long long>(mlen)));
   long long pb = P.pilot_min;
   if (P.pilot_den) {
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
     if (tid == 0) {
       P.pre_det[ns] = carry;
       P.gcnt[0] = 0u;
+      P.gcnt[1] = 0u;
     }
     return;
   }
@@ -242,7 +245,8 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   for (int i = tid; i < P.hist_words; i += blockDim.x) hist[i] = 0u;
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
   for (int i = tid; i < r.s1; i += blockDim.x) sel[i] = i;
-  for (int i = tid; i < n - r.wst; i += blockDim.x) sel[r.s1 + r.k + i] = r.wst + i;
+  if (P.topp_den == 0)  // with top-p, k_topp writes the window once k is known
+    for (int i = tid; i < n - r.wst; i += blockDim.x) sel[r.s1 + r.k + i] = r.wst + i;
 }
 
 // ============================================================ score pass helpers
@@ -1184,6 +1188,231 @@ __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, cons
     P.sel_count[u] = inf.nI + bsz;
   }
   __syncthreads();
+}
+
+// ============================================================ k_topp
+// Top-p selection (the mass-threshold variant of the predicted top-k): for
+// each unit, the number kk of highest-ranked middle positions (ranking key
+// order, ties to the lower position) whose share of the middle's softmax mass
+// under the scaled ranking scores first reaches p = topp_num / topp_den. Mass
+// in 2^-32 fixed point, w_j = rint(vexp(fl(r_j c) - max fl(r c)) 2^32), so the
+// cut is the exact integer test prefix * den >= num * S. The cut key comes
+// from a weighted radix select (digits of 11, 11 and 10 bits; u64 bin masses,
+// u128 comparisons); the keys equal to it all weigh the same, so the number
+// of them taken is the smallest m with (mass above + m w) * den >= num * S.
+// Writes the unit's k (and the regions that follow from it) and its window
+// positions; the last CTA then rebuilds the det gather's slice prefix. The
+// count-based select that follows takes exactly those kk keys. One CTA per
+// unit, keys read from L2 (the score pass wrote them just before).
+constexpr int kToppThreads = 1024;
+
+// fp32 value of an order key (inverse of ord_key; -0 comes back as +0).
+__device__ __forceinline__ float key_value(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__device__ __forceinline__ bool u128_ge(U128 a, U128 b) { return a.hi != b.hi ? a.hi > b.hi : a.lo >= b.lo; }
+__device__ __forceinline__ U128 mul_u64(unsigned long long a, unsigned long long b) {
+  return U128{a * b, __umul64hi(a, b)};
+}
+
+// Inclusive prefix sum of a u64 over the block (blockDim.x a multiple of 32).
+__device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* s_w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) s_w[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = lane < nw ? s_w[lane] : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    if (lane < nw) s_w[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long base = warp > 0 ? s_w[warp - 1] : 0ull;
+  __syncthreads();
+  return v + base;
+}
+
+// Over NB weighted bins (masses hm, counts hc), scanned from the top bin down:
+// the bin where (base + cumulative mass) * den first reaches target. Adds the
+// mass and count of the bins above it to *s_base / *s_cnt and writes the bin.
+template <int NB>
+__device__ void find_mass_digit(const unsigned long long* hm, const unsigned* hc, unsigned den, U128 target,
+                                unsigned long long* s_base, unsigned* s_cnt, int* s_digit,
+                                unsigned long long* s_w, unsigned* s_wc) {
+  constexpr int PER = NB / kToppThreads > 0 ? NB / kToppThreads : 1;
+  const int t = threadIdx.x;
+  const bool owns = (t + 1) * PER <= NB;
+  const int lo = owns ? NB - (t + 1) * PER : 0;  // bins [lo, lo + PER), scanned downwards
+  unsigned long long m = 0;
+  unsigned c = 0;
+  if (owns)
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+      m += hm[lo + i];
+      c += hc[lo + i];
+    }
+  const unsigned long long base = *s_base;
+  const unsigned cbase = *s_cnt;
+  const unsigned long long incl = block_scan_u64(m, s_w);
+  const unsigned cincl = block_inclusive_scan(c, s_wc);
+  const unsigned long long excl = incl - m;
+  const unsigned cexcl = cincl - c;
+  __syncthreads();  // every thread read s_base and s_cnt
+  if (owns && u128_ge(mul_u64(base + incl, den), target) && !u128_ge(mul_u64(base + excl, den), target)) {
+    unsigned long long acc = base + excl;
+    unsigned cacc = cbase + cexcl;
+    for (int i = PER - 1; i >= 0; i--) {
+      if (u128_ge(mul_u64(acc + hm[lo + i], den), target)) {
+        *s_digit = lo + i;
+        *s_base = acc;
+        *s_cnt = cacc;
+        break;
+      }
+      acc += hm[lo + i];
+      cacc += hc[lo + i];
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kToppThreads, 1) k_topp(DevParams P) {
+  __shared__ unsigned long long s_hm[kHist1];
+  __shared__ unsigned s_hc[kHist1];
+  __shared__ unsigned long long s_w[32];
+  __shared__ unsigned s_wc[32];
+  __shared__ unsigned long long s_base;
+  __shared__ unsigned s_cnt, s_kmax;
+  __shared__ int s_digit, s_last;
+  __shared__ long long s_carry;
+  const int u = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+  grid_dependency_wait();
+  const UnitInfo inf = P.info[u];
+  const int mlen = inf.wst - inf.s1;
+  const unsigned* keys = P.ordk + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+  const unsigned num = static_cast<unsigned>(P.topp_num), den = static_cast<unsigned>(P.topp_den);
+  int kk = 0;
+  if (inf.n > 0 && mlen > 0 && num > 0) {
+    // the largest ranking score of the middle
+    unsigned mk = 0;
+    for (int x = tid; x < mlen; x += nt) mk = max(mk, __ldcg(keys + x));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+    if (tid == 0) s_kmax = 0u;
+    __syncthreads();
+    if ((tid & 31) == 0) atomicMax(&s_kmax, mk);
+    __syncthreads();
+    const float smax = __fmul_rn(key_value(s_kmax), P.scale);
+    auto weight = [&](unsigned key) -> unsigned long long {
+      const float x = vexp(__fsub_rn(__fmul_rn(key_value(key), P.scale), smax));
+      return __float2ull_rn(__fmul_rn(x, 4294967296.0f));
+    };
+    // digit 1 masses and counts, and the total mass S
+    for (int i = tid; i < kHist1; i += nt) {
+      s_hm[i] = 0ull;
+      s_hc[i] = 0u;
+    }
+    if (tid == 0) {
+      s_base = 0ull;
+      s_cnt = 0u;
+      s_digit = 0;
+    }
+    __syncthreads();
+    unsigned long long tot = 0;
+    for (int x = tid; x < mlen; x += nt) {
+      const unsigned key = __ldcg(keys + x);
+      const unsigned long long w = weight(key);
+      tot += w;
+      atomicAdd(&s_hm[key >> 21], w);
+      atomicAdd(&s_hc[key >> 21], 1u);
+    }
+    const unsigned long long S = block_scan_u64(tot, s_w);  // the last thread holds the total
+    __shared__ unsigned long long s_S;
+    if (tid == nt - 1) s_S = S;
+    __syncthreads();
+    const U128 target = mul_u64(s_S, num);
+    find_mass_digit<kHist1>(s_hm, s_hc, den, target, &s_base, &s_cnt, &s_digit, s_w, s_wc);
+    const unsigned d1 = static_cast<unsigned>(s_digit);
+    // digit 2 within bin d1
+    for (int i = tid; i < kHist2; i += nt) {
+      s_hm[i] = 0ull;
+      s_hc[i] = 0u;
+    }
+    __syncthreads();
+    for (int x = tid; x < mlen; x += nt) {
+      const unsigned key = __ldcg(keys + x);
+      if ((key >> 21) == d1) {
+        atomicAdd(&s_hm[(key >> 10) & 2047u], weight(key));
+        atomicAdd(&s_hc[(key >> 10) & 2047u], 1u);
+      }
+    }
+    __syncthreads();
+    find_mass_digit<kHist2>(s_hm, s_hc, den, target, &s_base, &s_cnt, &s_digit, s_w, s_wc);
+    const unsigned pre = d1 << 11 | static_cast<unsigned>(s_digit);
+    // digit 3 within (d1, d2)
+    for (int i = tid; i < kHist3; i += nt) {
+      s_hm[i] = 0ull;
+      s_hc[i] = 0u;
+    }
+    __syncthreads();
+    for (int x = tid; x < mlen; x += nt) {
+      const unsigned key = __ldcg(keys + x);
+      if ((key >> 10) == pre) {
+        atomicAdd(&s_hm[key & 1023u], weight(key));
+        atomicAdd(&s_hc[key & 1023u], 1u);
+      }
+    }
+    __syncthreads();
+    find_mass_digit<kHist3>(s_hm, s_hc, den, target, &s_base, &s_cnt, &s_digit, s_w, s_wc);
+    // the cut key: keys above it are all taken; of the tied ones, the fewest
+    // (lowest positions first) that reach the target
+    if (tid == 0) {
+      const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
+      const unsigned long long wt = weight(thr);
+      unsigned lo = 1, hi = s_hc[s_digit];
+      while (lo < hi) {
+        const unsigned mid = lo + (hi - lo) / 2;
+        if (u128_ge(mul_u64(s_base + static_cast<unsigned long long>(mid) * wt, den), target))
+          hi = mid;
+        else
+          lo = mid + 1;
+      }
+      s_cnt += lo;
+    }
+    __syncthreads();
+    kk = static_cast<int>(s_cnt);
+  }
+  // the unit's regions with k = kk, and its window positions
+  const int ntail = mlen - kk;
+  const int nI = inf.s1 + kk + (inf.n - inf.wst);
+  if (tid == 0) {
+    P.info[u].k = kk;
+    P.info[u].ntail = ntail;
+    P.info[u].nI = nI;
+    P.info[u].nitems = nI;
+    P.info[u].mode = ntail == 0 ? 0 : (ntail <= inf.p ? 1 : 2);
+  }
+  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
+  for (int i = tid; i < inf.n - inf.wst; i += nt) sel[inf.s1 + kk + i] = inf.wst + i;
+  // the det gather's slice prefix follows from every unit's new state: the
+  // last CTA to get here rebuilds it
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(P.gcnt + 1, 1u) == static_cast<unsigned>(P.units - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    write_slice_prefix<kModeDet>(P, P.pre_det, s_wc, &s_carry);
+  }
+  grid_dependents_launch();
 }
 
 // Max score per head over unit u's det records (both parts) into s_mh.

@@ -60,7 +60,7 @@ class Workload:
     recipe: str
     guarantee: str = "denominator"  # "denominator" | "output": what the budget bounds
     topp_num: int = 0       # topp_den > 0: top-p selection, p = topp_num / topp_den
-    topp_den: int = 0       #   (the oracle only; the CUDA library selects a fixed k)
+    topp_den: int = 0
 
     @property
     def pages_per_seq(self):
