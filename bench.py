@@ -11,7 +11,9 @@ and larger than L2 (so no flush is needed). Prints one JSON line (rank 0).
 The headline is --workload (default gqa_32k); at one GPU the line also carries
 `per_config`, the same measurements for the other long-context workloads
 (sparq_128k, loki_64k, paged_sweep at eps 0.05). The score pass's roofline is
-timed by events on SCORE_SAMPLES further calls after the timed region.
+timed by events on SCORE_SAMPLES further calls after the timed region. `host_kv`
+times the HOST_KV workloads with their K and V caches in page-locked host memory,
+against dense decode over the same host-resident caches.
 Under torchrun each rank runs its own batch on its own GPU (weak scaling; no
 collective on the data path, one max-reduction of the elapsed time).
 """
@@ -38,6 +40,8 @@ NOMINAL_HBM_GBS = 8000.0
 SCORE_SAMPLES = 64   # score passes timed by events after the timed region
 # the other long-context workloads measured in the same run (name, eps override)
 PER_CONFIG = [("sparq_128k", None), ("loki_64k", None), ("paged_sweep", 0.05)]
+# workloads also timed with their K and V caches in page-locked host memory
+HOST_KV = ["loki_64k"]
 KERNEL_SOURCE = "verified_sparse_attention_b200/csrc/vattn_kernels.cuh"
 # the sections of KERNEL_SOURCE that hold the ranking-score pass (its kernels
 # and their own helpers): the DRAM counters in profiles/ are keyed to them
@@ -306,6 +310,55 @@ def run_e2e(args, w, x, dec, prm, stream, dev, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
+def run_host_kv(name, args, dev):
+    """Workload `name` with its K and V caches in page-locked host memory (the proxy
+    caches, q, page table and lengths on the GPU): sparse calls/s against dense decode
+    over the same host-resident caches, both by CUDA events on the launching stream."""
+    w = synth.WORKLOADS[name]
+    xd = synth.make_inputs(w, device=dev)
+    x = dict(xd, k_cache=xd["k_cache"].cpu().pin_memory(), v_cache=xd["v_cache"].cpu().pin_memory())
+    del xd
+    torch.cuda.empty_cache()
+    dec = decoder_for(w, device=dev, kv_location="host")
+    prm = params_for(w, x)
+    outs = dec.alloc_outputs(w.batch)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    sparse_ms = timed(lambda: dec.decode(x["q"], x["k_cache"], x["v_cache"], x["page_table"],
+                                         x["seq_lens"], prm, outputs=outs, stream=stream),
+                      args.host_kv_steps)
+    if dec.last_error():
+        raise RuntimeError(f"{name} (host-resident caches): device error word set")
+    dense_ms = timed(lambda: dec.dense(x["q"], x["k_cache"], x["v_cache"], x["page_table"],
+                                       x["seq_lens"], x["num_pages"], stream=stream),
+                     max(1, args.host_kv_steps // 4))
+    b = algorithmic_bytes(w, x, outs)
+    e = synth.bytes_per_elem(w)
+    host_sparse = b["gather"] + (b["score_read"] if w.proxy == "exact" else 0)
+    host_dense = int(x["seq_lens"].to(torch.int64).sum()) * w.num_kv_heads * 2 * w.head_dim * e
+    dec.close()
+    del x
+    torch.cuda.empty_cache()
+    return {"workload": synth.describe(w), "calls_per_s": 1e3 / sparse_ms,
+            "dense_calls_per_s": 1e3 / dense_ms, "speedup_vs_dense": dense_ms / sparse_ms,
+            "host_bytes_per_call": host_sparse, "dense_host_bytes_per_call": host_dense,
+            "host_link_gbs": host_sparse / (sparse_ms / 1e3) / 1e9,
+            "dense_host_link_gbs": host_dense / (dense_ms / 1e3) / 1e9,
+            "steps": args.host_kv_steps}
+
+
 def time_oracle_all_cores(w, cpu_inputs, budget_s):
     """The same oracle on every host core: one thread per core, each running whole
     (sequence, KV head) units (the C library releases the GIL) until budget_s.
@@ -372,6 +425,8 @@ def main():
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other long-context workloads")
     ap.add_argument("--per-config-steps", type=int, default=200)
+    ap.add_argument("--host-kv-steps", type=int, default=8,
+                    help="decode calls timed with the KV cache in host memory (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -475,6 +530,8 @@ def main():
             del x_c, dec_c
             torch.cuda.empty_cache()
         line["per_config"] = per
+    if world == 1 and args.host_kv_steps > 0 and args.guarantee == "denominator":
+        line["host_kv"] = {name: run_host_kv(name, args, dev) for name in HOST_KV}
     if ranks.reports(rank):
         emit(line)
     if world > 1:

@@ -81,6 +81,8 @@ extern "C" {
 
 enum { VATTN_FP32 = 0, VATTN_BF16 = 1 };
 enum { VATTN_EXACT = 0, VATTN_SPARQ = 1, VATTN_LOKI = 2 };
+/* where the K and V caches live (vattn_config.kv_location) */
+enum { VATTN_KV_DEVICE = 0, VATTN_KV_HOST = 1 };
 /* what the sample size bounds: the softmax denominator alone (the pages'
    practical form), or the denominator and the numerator vector (output) */
 enum { VATTN_GUARANTEE_DENOMINATOR = 0, VATTN_GUARANTEE_OUTPUT = 1 };
@@ -112,6 +114,17 @@ typedef struct {
   int max_ctx;      /* upper bound on seq_lens[b]; 1 <= max_ctx <= 2^24          */
   int proxy;        /* VATTN_EXACT, VATTN_SPARQ or VATTN_LOKI                    */
   int proxy_rank;   /* SparQ: r in [1, d]; Loki: the stored rank, 32             */
+  /* VATTN_KV_DEVICE: k_cache and v_cache are device memory. VATTN_KV_HOST: they
+     are page-locked host memory (cudaHostAlloc / cudaMallocHost, or
+     cudaHostRegister with cudaHostRegisterMapped), passed by their host
+     address; the library maps each call's pointers to their device addresses
+     and reads only the rows it selects (and, in exact mode, the whole of K for
+     the ranking pass) over the host link ("vAttention: A New Approach to
+     Sparse Attention with Guaranteed Accuracy", section "Performance and
+     Efficiency": speedups when the KV cache is hosted on the CPU). Every other
+     array, the SparQ and Loki proxy caches included, stays in device memory.
+     A cache pointer that is not page-locked host memory returns VATTN_EINVAL. */
+  int kv_location;
 } vattn_config;
 
 /* Per call. */

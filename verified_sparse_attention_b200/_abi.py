@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libvattn.so")
 
 VATTN_FP32, VATTN_BF16 = 0, 1
 VATTN_EXACT, VATTN_SPARQ, VATTN_LOKI = 0, 1, 2
+VATTN_KV_DEVICE, VATTN_KV_HOST = 0, 1
 VATTN_GUARANTEE_DENOMINATOR, VATTN_GUARANTEE_OUTPUT = 0, 1
 VATTN_OK, VATTN_EINVAL, VATTN_ENOMEM, VATTN_ECUDA, VATTN_ESCRATCH = 0, -1, -2, -3, -4
 VATTN_DEV_BAD_SEQLEN, VATTN_DEV_BAD_PAGE, VATTN_DEV_TIMEOUT = 1, 2, 4
@@ -27,7 +28,8 @@ EXPORTS = ("vattn_create", "vattn_decode", "vattn_dense_decode", "vattn_dense_de
 class vattn_config(C.Structure):
     _fields_ = [("num_q_heads", C.c_int), ("num_kv_heads", C.c_int), ("head_dim", C.c_int),
                 ("dtype", C.c_int), ("page_size", C.c_int), ("max_batch", C.c_int),
-                ("max_ctx", C.c_int), ("proxy", C.c_int), ("proxy_rank", C.c_int)]
+                ("max_ctx", C.c_int), ("proxy", C.c_int), ("proxy_rank", C.c_int),
+                ("kv_location", C.c_int)]
 
 
 class vattn_params(C.Structure):

@@ -204,6 +204,33 @@ int check_config(const vattn_config* c) {
   } else if (c->proxy != VATTN_EXACT) {
     return VATTN_EINVAL;
   }
+  if (c->kv_location != VATTN_KV_DEVICE && c->kv_location != VATTN_KV_HOST) return VATTN_EINVAL;
+  return VATTN_OK;
+}
+
+// Device address of a cache in page-locked host memory (nullptr if `p` is not
+// such memory).
+const void* host_cache_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  return static_cast<const char*>(a.devicePointer) +
+         (static_cast<const char*>(p) - static_cast<const char*>(a.hostPointer ? a.hostPointer : p));
+}
+
+// The caches as the kernels address them (host-resident caches mapped to
+// their device addresses); VATTN_EINVAL if a host-resident cache is not
+// page-locked.
+int cache_ptrs(const vattn_config& c, const void** k, const void** v) {
+  if (c.kv_location != VATTN_KV_HOST) return VATTN_OK;
+  const void* dk = host_cache_device_ptr(*k);
+  const void* dv = host_cache_device_ptr(*v);
+  if (!dk || !dv) return VATTN_EINVAL;
+  *k = dk;
+  *v = dv;
   return VATTN_OK;
 }
 
@@ -222,6 +249,7 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->units = batch * c.num_kv_heads;
   P->proxy = c.proxy;
   P->rank = c.proxy_rank;
+  P->kv_host = c.kv_location == VATTN_KV_HOST;
   P->scale = static_cast<float>(1.0 / sqrt(static_cast<double>(c.head_dim)));
   P->nseg = ctx->nseg;
   P->info = ctx->info;
@@ -315,7 +343,10 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score, 256, 0);
   ctx->score_grid = (occ < 1 ? 1 : occ) * ctx->num_sms;
-  if (cfg->page_size >= cfg->max_ctx && cfg->proxy != VATTN_SPARQ) {
+  // the bulk-copy score pass streams a contiguous cache in device memory (the
+  // proxy cache for Loki, K itself in exact mode)
+  if (cfg->page_size >= cfg->max_ctx && cfg->proxy != VATTN_SPARQ &&
+      (cfg->proxy == VATTN_LOKI || cfg->kv_location == VATTN_KV_DEVICE)) {
     void (*tma)(DevParams) = cfg->proxy == VATTN_LOKI ? K.score_loki_tma : K.score_exact_tma;
     const size_t smem = cfg->proxy == VATTN_LOKI ? K.score_loki_tma_smem : K.score_tma_smem;
     if (cudaFuncSetAttribute(tma, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
@@ -512,7 +543,10 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.guarantee = prm->guarantee == VATTN_GUARANTEE_OUTPUT;
   P.topp_num = prm->topp_num;
   P.topp_den = prm->topp_den;
-  if (const int rc = encode_row_maps(c, k_cache, v_cache, prm->num_pages, &P)) return ctx->last_status = rc;
+  if (const int rc = cache_ptrs(c, &k_cache, &v_cache)) return ctx->last_status = rc;
+  // row maps for the gathers' tensor copies (host-resident caches use plain loads)
+  if (!P.kv_host)
+    if (const int rc = encode_row_maps(c, k_cache, v_cache, prm->num_pages, &P)) return ctx->last_status = rc;
   P.q = q;
   P.k = k_cache;
   P.v = v_cache;
@@ -604,7 +638,9 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.pilot_min = 2;
   P.eps = 1.0f;
   P.num_pages = num_pages;
-  if (const int rc = encode_row_maps(c, k_cache, v_cache, num_pages, &P)) return ctx->last_status = rc;
+  if (const int rc = cache_ptrs(c, &k_cache, &v_cache)) return ctx->last_status = rc;
+  if (!P.kv_host)
+    if (const int rc = encode_row_maps(c, k_cache, v_cache, num_pages, &P)) return ctx->last_status = rc;
   P.proxy = VATTN_EXACT;
   P.q = q;
   P.k = k_cache;

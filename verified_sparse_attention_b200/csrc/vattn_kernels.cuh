@@ -885,6 +885,11 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
 __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Plain arrival (no transaction bytes): completes a phase whose stage was
+// filled by ordinary stores.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
@@ -1817,6 +1822,39 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(con
       // memory form runs (a lane starts one when its row does not directly
       // follow the previous lane's)
       int row = lane < nvalid ? (pid * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps) : 0;
+      if (P.kv_host) {
+        // caches in mapped host memory: the warp reads the block's rows with
+        // plain 16-byte loads over the host link (eight in flight per lane),
+        // stores them into the stage and completes its phase with a plain
+        // arrival; rows past the end are zero
+        constexpr int VPR = ROWB / 16;
+        constexpr int PER = R * VPR / 32;  // vectors of each matrix per lane
+        constexpr int CH = PER < 4 ? PER : 4;
+#pragma unroll
+        for (int i0 = 0; i0 < PER; i0 += CH) {
+          uint4 kx[CH], vx[CH];
+#pragma unroll
+          for (int i = 0; i < CH; i++) {
+            const int x = (i0 + i) * 32 + lane, r = x / VPR, cc = x % VPR;
+            const int rr = __shfl_sync(0xffffffffu, row, r);
+            kx[i] = vx[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < nvalid) {
+              const size_t off = static_cast<size_t>(rr) * D + cc * E;
+              kx[i] = ld_gather(kc + off);
+              vx[i] = ld_gather(vc + off);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < CH; i++) {
+            const int x = (i0 + i) * 32 + lane, r = x / VPR, cc = x % VPR;
+            *reinterpret_cast<uint4*>(dst + r * ROWB + cc * 16) = kx[i];
+            *reinterpret_cast<uint4*>(dst + (R + r) * ROWB + cc * 16) = vx[i];
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[st]);
+        return;
+      }
       const int prev = __shfl_up_sync(0xffffffffu, row, 1);
       const bool start = lane < nvalid && (lane == 0 || row != prev + 1);
       const unsigned starts = __ballot_sync(0xffffffffu, start);
@@ -2418,7 +2456,11 @@ __global__ void __launch_bounds__(kNumThreads) k_numstats(DevParams P) {
       unsigned char* dst = s_v + buf * kNumBufBytes;
       for (int x = tid; x < cnt * V16; x += kNumThreads) {
         const int i = x / V16, k = x % V16;
-        cp_async16(dst + i * ROWB + k * 16, vb + static_cast<size_t>(s_row[c0 + i]) * ROWB + k * 16);
+        const char* src = vb + static_cast<size_t>(s_row[c0 + i]) * ROWB + k * 16;
+        if (P.kv_host)  // mapped host memory: a plain load (the round's use waits on a barrier)
+          *reinterpret_cast<uint4*>(dst + i * ROWB + k * 16) = ld_gather(src);
+        else
+          cp_async16(dst + i * ROWB + k * 16, src);
       }
       const float* src = ps + static_cast<size_t>(s0 + c0) * G;
       for (int x = tid; x < cnt * G; x += kNumThreads) cp_async4(&s_ps[buf][x], src + x);

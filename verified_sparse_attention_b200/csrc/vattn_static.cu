@@ -364,6 +364,7 @@ extern "C" int vattn_dense_decode_static(const vattn_config* cfg, const void* q,
   if (c.max_batch < 1 || c.max_ctx < 1 || c.max_ctx > (1 << 24)) return VATTN_EINVAL;
   if (batch < 0 || batch > c.max_batch || num_pages < 1) return VATTN_EINVAL;
   if (!aligned16(k_cache) || !aligned16(v_cache)) return VATTN_EINVAL;
+  if (c.kv_location != VATTN_KV_DEVICE && c.kv_location != VATTN_KV_HOST) return VATTN_EINVAL;
   const long long units = static_cast<long long>(batch) * c.num_kv_heads;
   const size_t rec_bytes = static_cast<size_t>(G) * (c.head_dim + 2) * sizeof(float);
   if (static_cast<size_t>(units) * rec_bytes > kStaticScratchBytes) return VATTN_ESCRATCH;
@@ -372,6 +373,19 @@ extern "C" int vattn_dense_decode_static(const vattn_config* cfg, const void* q,
   DeviceSlot slot;
   const int rc = device_slot(&slot);
   if (rc != VATTN_OK) return rc;
+  if (c.kv_location == VATTN_KV_HOST) {  // page-locked host caches: their device addresses
+    cudaPointerAttributes ak, av;
+    if (cudaPointerGetAttributes(&ak, k_cache) != cudaSuccess || cudaPointerGetAttributes(&av, v_cache) != cudaSuccess) {
+      cudaGetLastError();
+      return VATTN_EINVAL;
+    }
+    if (ak.type != cudaMemoryTypeHost || av.type != cudaMemoryTypeHost || !ak.devicePointer || !av.devicePointer)
+      return VATTN_EINVAL;
+    k_cache = static_cast<const char*>(ak.devicePointer) +
+              (static_cast<const char*>(k_cache) - static_cast<const char*>(ak.hostPointer ? ak.hostPointer : k_cache));
+    v_cache = static_cast<const char*>(av.devicePointer) +
+              (static_cast<const char*>(v_cache) - static_cast<const char*>(av.hostPointer ? av.hostPointer : v_cache));
+  }
   SplitFn split;
   MergeFn merge;
   if (!pick(c, G, &split, &merge)) return VATTN_EINVAL;

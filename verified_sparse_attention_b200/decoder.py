@@ -10,13 +10,15 @@ from . import _abi
 _DTYPES = {torch.float32: _abi.VATTN_FP32, torch.bfloat16: _abi.VATTN_BF16}
 _PROXIES = {"exact": _abi.VATTN_EXACT, "sparq": _abi.VATTN_SPARQ, "loki": _abi.VATTN_LOKI}
 _GUARANTEES = {"denominator": _abi.VATTN_GUARANTEE_DENOMINATOR, "output": _abi.VATTN_GUARANTEE_OUTPUT}
+# "host": k_cache and v_cache are page-locked host tensors (tensor.pin_memory())
+_KV = {"device": _abi.VATTN_KV_DEVICE, "host": _abi.VATTN_KV_HOST}
 
 
 class SparseDecoder:
     """A vattn context for fixed shapes (see vattn_config in include/vattn.h)."""
 
     def __init__(self, *, num_q_heads, num_kv_heads, head_dim, dtype, page_size, max_batch,
-                 max_ctx, proxy="exact", proxy_rank=0, device=None):
+                 max_ctx, proxy="exact", proxy_rank=0, device=None, kv_location="device"):
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.max_batch, self.max_ctx, self.page_size = max_batch, max_ctx, page_size
@@ -25,7 +27,7 @@ class SparseDecoder:
         cfg = _abi.vattn_config(num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
                                 head_dim=head_dim, dtype=_DTYPES[dtype], page_size=page_size,
                                 max_batch=max_batch, max_ctx=max_ctx, proxy=_PROXIES[proxy],
-                                proxy_rank=proxy_rank)
+                                proxy_rank=proxy_rank, kv_location=_KV[kv_location])
         with torch.cuda.device(self.device):
             self.ctx = _abi.vattn_create(cfg)
 
@@ -84,13 +86,14 @@ class SparseDecoder:
             pass
 
 
-def decoder_for(w, device=None, max_batch=None):
+def decoder_for(w, device=None, max_batch=None, kv_location="device"):
     """A SparseDecoder shaped for a synthetic workload description (synth.Workload)."""
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     return SparseDecoder(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                          head_dim=w.head_dim, dtype=dt, page_size=w.page_size,
                          max_batch=w.batch if max_batch is None else max_batch, max_ctx=w.max_ctx,
-                         proxy=w.proxy, proxy_rank=w.proxy_rank, device=device)
+                         proxy=w.proxy, proxy_rank=w.proxy_rank, device=device,
+                         kv_location=kv_location)
 
 
 def params_for(w, inputs, eps=None, seed=None, guarantee=None):
