@@ -15,7 +15,9 @@ timed by events on SCORE_SAMPLES further calls after the timed region. `host_kv`
 times the HOST_KV workloads with their K and V caches in page-locked host memory,
 against dense decode over the same host-resident caches.
 Under torchrun each rank runs its own batch on its own GPU (weak scaling; no
-collective on the data path, one max-reduction of the elapsed time).
+collective on the data path, one max-reduction of the elapsed time); with
+--shard heads|batch the ranks split one batch instead and all-gather its
+outputs over NCCL in every step (strong scaling).
 """
 import argparse
 import hashlib
@@ -359,6 +361,48 @@ def run_host_kv(name, args, dev):
             "steps": args.host_kv_steps}
 
 
+def run_sharded(args, w, rank, world, dev):
+    """One batch split over the ranks (--shard heads|batch): each rank decodes its slice
+    and the outputs are all-gathered over NCCL inside every timed step, so a step is
+    one whole-batch call (strong scaling)."""
+    x = synth.make_inputs(w, device=dev)  # the whole batch (same seed on every rank)
+    ws, boff, hoff = ranks.shard_workload(w, args.shard, world, rank)
+    xs = ranks.shard_inputs(x, w, args.shard, world, rank)
+    del x
+    torch.cuda.empty_cache()
+    dec = decoder_for(ws, device=dev)
+    prm = params_for(ws, xs, batch_offset=boff, head_offset=hoff)
+    outs = dec.alloc_outputs(ws.batch)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dec.decode(xs["q"], xs["k_cache"], xs["v_cache"], xs["page_table"], xs["seq_lens"], prm,
+                   outputs=outs, stream=stream)
+        return ranks.gather_outputs(outs, args.shard, world)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dec.last_error():
+        raise RuntimeError("device error word set during warm-up")
+    ranks.barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ranks.barrier(world)
+    ms = ranks.max_over_ranks(a.elapsed_time(b), world, dev)
+    launches = _abi.vattn_last_launch_count(dec.ctx) * args.steps
+    dec.close()
+    return {"value": args.steps / (ms / 1e3), "ms": ms, "clocks": clk.summary(), "gpu_launches": launches,
+            "shard": {"mode": args.shard, "units_per_rank": ws.units, "units": w.units,
+                      "collective": "all_gather of out, sel_idx, sel_count, budgets, head_need"}}
+
+
 def time_oracle_all_cores(w, cpu_inputs, budget_s):
     """The same oracle on every host core: one thread per core, each running whole
     (sequence, KV head) units (the C library releases the GIL) until budget_s.
@@ -425,6 +469,9 @@ def main():
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other long-context workloads")
     ap.add_argument("--per-config-steps", type=int, default=200)
+    ap.add_argument("--shard", default=None, choices=list(ranks.SHARD_MODES),
+                    help="split one batch over the ranks (by KV head or by sequence) and "
+                         "all-gather the outputs, instead of one batch per rank")
     ap.add_argument("--host-kv-steps", type=int, default=8,
                     help="decode calls timed with the KV cache in host memory (0: skip)")
     args = ap.parse_args()
@@ -471,6 +518,19 @@ def main():
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peak, peak_kind = load_peaks()
+    if args.shard:
+        r = run_sharded(args, w, rank, world, dev)
+        cfg["parallelism"] = f"shard-{args.shard}{world}"
+        if ranks.reports(rank):
+            emit({"metric": METRIC, "value": r["value"], "unit": "calls/s", "n_gpus": world,
+                  "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
+                  "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                  "dtype": w.dtype, "data": "synthetic", "config": cfg, "shard": r["shard"],
+                  "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]})
+        if world > 1:
+            ranks.barrier(world)
+            torch.distributed.destroy_process_group()
+        return
     wr = ranks.rank_workload(w, rank)
     dec, x, prm, r = run_config(wr, args, dev, world, args.steps, headline=True)
     sm = summarize(r, world, peak)

@@ -159,6 +159,13 @@ typedef struct {
      budget's fixed-order exp) so that the cut is the exact integer test
      prefix * den >= num * S. 0 <= topp_num <= topp_den; topp_den = 0: off. */
   int topp_num, topp_den;
+  /* Sharded runs: when this call decodes a slice of a larger batch (a range of
+     sequences, or a range of KV heads with their query heads), the index of its
+     first sequence and first KV head in the whole batch. The sampler's draw
+     counter names the sequence and KV head in the whole batch, (batch_offset + b,
+     head_offset + h), so the shards together draw exactly what one call over the
+     whole batch would. 0 for an unsharded call; both >= 0. */
+  int batch_offset, head_offset;
 } vattn_params;
 
 /* Create a context on the current CUDA device and allocate its workspace.

@@ -34,6 +34,7 @@ class Problem(C.Structure):
         ("eps", C.c_float), ("delta", C.c_float), ("seed", C.c_uint64),
         ("guarantee", C.c_int),
         ("topp_num", C.c_int), ("topp_den", C.c_int),
+        ("batch_offset", C.c_int), ("head_offset", C.c_int),
     ]
 
 
@@ -128,10 +129,11 @@ def ord_key(f, L=None):
     return (L or lib()).orc_ord(float(f))
 
 
-def make_problem(w, seed=None, eps=None, batch=None, guarantee=None):
+def make_problem(w, seed=None, eps=None, batch=None, guarantee=None, batch_offset=0, head_offset=0):
     """Problem struct from a workload description (verified_sparse_attention_b200.synth.Workload).
 
-    `guarantee` ("denominator" or "output") overrides the workload's own.
+    `guarantee` ("denominator" or "output") overrides the workload's own; the
+    offsets place a shard of a larger batch (its first sequence and KV head).
     """
     return Problem(
         batch=batch if batch is not None else w.batch, num_q_heads=w.num_q_heads,
@@ -143,7 +145,8 @@ def make_problem(w, seed=None, eps=None, batch=None, guarantee=None):
         eps=w.eps if eps is None else eps, delta=w.delta,
         seed=w.seed if seed is None else seed,
         guarantee=GUARANTEES[guarantee or getattr(w, "guarantee", "denominator")],
-        topp_num=getattr(w, "topp_num", 0), topp_den=getattr(w, "topp_den", 0))
+        topp_num=getattr(w, "topp_num", 0), topp_den=getattr(w, "topp_den", 0),
+        batch_offset=batch_offset, head_offset=head_offset)
 
 
 def decode(problem, inputs, units=None, L=None):

@@ -63,6 +63,7 @@ typedef struct {
   uint64_t seed;
   int guarantee; /* ORC_GUARANTEE_DENOMINATOR or ORC_GUARANTEE_OUTPUT */
   int topp_num, topp_den; /* topp_den > 0: top-p selection with p = topp_num / topp_den */
+  int batch_offset, head_offset; /* a shard's first sequence and KV head in the whole batch */
 } orc_problem;
 
 /* ------------------------------------------------------------------ */
@@ -92,7 +93,9 @@ void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint3
 }
 
 /* Draw t of unit (b, h): counter (t/4, b, h, 0), key = the 64-bit seed split */
-/* into (low word, high word); the draw is word t%4 of that block.           */
+/* into (low word, high word); the draw is word t%4 of that block. b and h   */
+/* name the sequence and KV head in the whole batch: a shard of a batch adds */
+/* its offsets, so that the shards draw what the whole batch would.          */
 uint32_t orc_draw_word(uint64_t seed, uint32_t b, uint32_t h, uint32_t t) {
   uint32_t ctr[4] = {t >> 2, b, h, 0u};
   uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
@@ -413,7 +416,7 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
   } else {
     int32_t* pil = malloc(sizeof(int32_t) * (size_t)p);
     for (int t = 0; t < p; t++) {
-      uint32_t u = orc_draw_word(pr->seed, (uint32_t)b, (uint32_t)h, (uint32_t)t);
+      uint32_t u = orc_draw_word(pr->seed, (uint32_t)(b + pr->batch_offset), (uint32_t)(h + pr->head_offset), (uint32_t)t);
       uint32_t rho = (uint32_t)(((uint64_t)u * (uint64_t)ntail) >> 32);
       pil[t] = tail[rho];
     }
@@ -533,7 +536,7 @@ static void decode_unit(const orc_problem* pr, const orc_inputs* in, const orc_o
     for (int t = 0; t < ntail; t++) sel[nI + t] = tail[t];
   } else if (ntail > 0) {
     for (int t = 0; t < bsz; t++) {
-      uint32_t u = orc_draw_word(pr->seed, (uint32_t)b, (uint32_t)h, (uint32_t)t);
+      uint32_t u = orc_draw_word(pr->seed, (uint32_t)(b + pr->batch_offset), (uint32_t)(h + pr->head_offset), (uint32_t)t);
       uint32_t rho = (uint32_t)(((uint64_t)u * (uint64_t)ntail) >> 32);
       sel[nI + t] = tail[rho];
     }
@@ -605,6 +608,7 @@ int orc_decode(const orc_problem* pr, const void* q, const void* k_cache, const 
   if (pr->pilot_min < 2) return -1;
   if (pr->guarantee != ORC_GUARANTEE_DENOMINATOR && pr->guarantee != ORC_GUARANTEE_OUTPUT) return -1;
   if (pr->topp_den < 0 || pr->topp_num < 0 || (pr->topp_den > 0 && pr->topp_num > pr->topp_den)) return -1;
+  if (pr->batch_offset < 0 || pr->head_offset < 0) return -1;
   if (pr->sinks < 0 || pr->window < 0 || pr->topk_abs < 0 || pr->topk_num < 0 || pr->topk_den < 0 ||
       pr->pilot_num < 0 || pr->pilot_den < 0)
     return -1;

@@ -39,7 +39,8 @@ class vattn_params(C.Structure):
                 ("eps", C.c_float), ("delta", C.c_float), ("seed", C.c_uint64),
                 ("num_pages", C.c_int),
                 ("k_t_cache", C.c_void_p), ("k_proj_cache", C.c_void_p), ("proj_basis", C.c_void_p),
-                ("guarantee", C.c_int), ("topp_num", C.c_int), ("topp_den", C.c_int)]
+                ("guarantee", C.c_int), ("topp_num", C.c_int), ("topp_den", C.c_int),
+                ("batch_offset", C.c_int), ("head_offset", C.c_int)]
 
 
 class VattnError(RuntimeError):

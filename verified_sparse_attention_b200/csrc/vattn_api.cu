@@ -511,6 +511,7 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   if (prm->guarantee != VATTN_GUARANTEE_DENOMINATOR && prm->guarantee != VATTN_GUARANTEE_OUTPUT)
     return VATTN_EINVAL;
   if (prm->topp_den < 0 || prm->topp_num < 0 || prm->topp_num > prm->topp_den) return VATTN_EINVAL;
+  if (prm->batch_offset < 0 || prm->head_offset < 0) return VATTN_EINVAL;
   if (c.proxy == VATTN_SPARQ && (!prm->k_t_cache || !aligned16(prm->k_t_cache))) return VATTN_EINVAL;
   if (c.proxy == VATTN_LOKI && (!prm->k_proj_cache || !prm->proj_basis || !aligned16(prm->k_proj_cache)))
     return VATTN_EINVAL;
@@ -543,6 +544,8 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.guarantee = prm->guarantee == VATTN_GUARANTEE_OUTPUT;
   P.topp_num = prm->topp_num;
   P.topp_den = prm->topp_den;
+  P.batch_offset = prm->batch_offset;
+  P.head_offset = prm->head_offset;
   if (const int rc = cache_ptrs(c, &k_cache, &v_cache)) return ctx->last_status = rc;
   // row maps for the gathers' tensor copies (host-resident caches use plain loads)
   if (!P.kv_host)

@@ -65,6 +65,7 @@ struct DevParams {
   int guarantee;    // 1: the budget also bounds the numerator vector (output guarantee)
   int topp_num, topp_den;  // topp_den > 0: top-p selection with p = topp_num / topp_den
   int kv_host;      // 1: k and v point into mapped host memory (plain loads only)
+  int batch_offset, head_offset;  // a shard's first sequence and KV head in the whole batch
   int CD, CS;       // grid sizes of the det (and dense) and sample gathers
   // inputs
   const void* q;

@@ -2100,7 +2100,10 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
     topk = s_topk;
   }
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
-  const unsigned bb = static_cast<unsigned>(u / P.Hkv), hh = static_cast<unsigned>(u % P.Hkv);
+  // the draw counter names the sequence and KV head in the whole batch (a
+  // shard adds its offsets), so a shard draws what the whole batch would
+  const unsigned bb = static_cast<unsigned>(P.batch_offset + u / P.Hkv),
+                 hh = static_cast<unsigned>(P.head_offset + u % P.Hkv);
   const int step0 = inf.k > 0 ? 1 << (31 - __clz(inf.k)) : 0;
   // each thread takes aligned groups of four draws: one Philox block serves
   // all four, and their four searches advance together
@@ -2312,7 +2315,10 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
   const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
   const bool whole = inf.mode == 1;
   int* dsel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
-  const unsigned bb = static_cast<unsigned>(u / P.Hkv), hh = static_cast<unsigned>(u % P.Hkv);
+  // the draw counter names the sequence and KV head in the whole batch (a
+  // shard adds its offsets), so a shard draws what the whole batch would
+  const unsigned bb = static_cast<unsigned>(P.batch_offset + u / P.Hkv),
+                 hh = static_cast<unsigned>(P.head_offset + u % P.Hkv);
   for (int t = tid; t < t1; t += kSel1Threads) {
     const int rho = whole ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
     dsel[t] = tail_position(topk, inf.k, inf.s1, rho);

@@ -44,7 +44,7 @@ class SparseDecoder:
     def make_params(*, sinks, window, topk_abs=0, topk_num=0, topk_den=0, pilot_min=64,
                     pilot_num=0, pilot_den=0, eps, delta, seed, num_pages, k_t_cache=None,
                     k_proj_cache=None, proj_basis=None, guarantee="denominator", topp_num=0,
-                    topp_den=0):
+                    topp_den=0, batch_offset=0, head_offset=0):
         return _abi.vattn_params(
             sinks=sinks, window=window, topk_abs=topk_abs, topk_num=topk_num, topk_den=topk_den,
             pilot_min=pilot_min, pilot_num=pilot_num, pilot_den=pilot_den, eps=eps, delta=delta,
@@ -52,7 +52,8 @@ class SparseDecoder:
             k_t_cache=None if k_t_cache is None else k_t_cache.data_ptr(),
             k_proj_cache=None if k_proj_cache is None else k_proj_cache.data_ptr(),
             proj_basis=None if proj_basis is None else proj_basis.data_ptr(),
-            guarantee=_GUARANTEES[guarantee], topp_num=topp_num, topp_den=topp_den)
+            guarantee=_GUARANTEES[guarantee], topp_num=topp_num, topp_den=topp_den,
+            batch_offset=batch_offset, head_offset=head_offset)
 
     def decode(self, q, k_cache, v_cache, page_table, seq_lens, params, outputs=None, stream=None):
         batch = q.shape[0]
@@ -96,12 +97,14 @@ def decoder_for(w, device=None, max_batch=None, kv_location="device"):
                          kv_location=kv_location)
 
 
-def params_for(w, inputs, eps=None, seed=None, guarantee=None):
-    """vattn_params of a synthetic workload with its drawn inputs (device tensors)."""
+def params_for(w, inputs, eps=None, seed=None, guarantee=None, batch_offset=0, head_offset=0):
+    """vattn_params of a synthetic workload with its drawn inputs (device tensors); the
+    offsets place a shard of a larger batch."""
     return SparseDecoder.make_params(
         sinks=w.sinks, window=w.window, topk_abs=w.topk_abs, topk_num=w.topk_num,
         topk_den=w.topk_den, pilot_min=w.pilot_min, pilot_num=w.pilot_num, pilot_den=w.pilot_den,
         eps=w.eps if eps is None else eps, delta=w.delta, seed=w.seed if seed is None else seed,
         num_pages=int(inputs["num_pages"]), k_t_cache=inputs.get("k_t_cache"),
         k_proj_cache=inputs.get("k_proj_cache"), proj_basis=inputs.get("proj_basis"),
-        guarantee=guarantee or w.guarantee, topp_num=w.topp_num, topp_den=w.topp_den)
+        guarantee=guarantee or w.guarantee, topp_num=w.topp_num, topp_den=w.topp_den,
+        batch_offset=batch_offset, head_offset=head_offset)
