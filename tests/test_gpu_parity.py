@@ -114,14 +114,28 @@ def test_dtype_and_head_dim(dtype, d):
     check(w)
 
 
-def test_long_max_ctx_uses_grid_wide_selection():
-    # a context bound whose per-CTA key segment does not fit in shared memory
-    # selects the top-k with the grid-wide passes instead of one cluster per unit
+def test_long_max_ctx_streams_the_keys():
+    # a context bound whose keys do not fit one CTA's shared memory selects with
+    # k_topk, which streams the keys from L2
     small = synth.scaled(W["gqa_32k"], max_ctx=9000, batch=1, num_q_heads=8, num_kv_heads=2)
     cpu = synth.make_inputs(small)
     w = small.replace(max_ctx=600000, min_ctx=600000)      # same page size, longer bound
     pad = torch.full((1, w.pages_per_seq - cpu["page_table"].shape[1]), -1, dtype=torch.int32)
     cpu["page_table"] = torch.cat([cpu["page_table"], pad], 1)
+    check(w, inputs=cpu)
+
+
+@pytest.mark.parametrize("case", ["equal_scores", "k_above_list_space", "planted"])
+def test_streamed_select_at_long_context(case):
+    # k_topk (middles longer than one CTA's shared memory): the single ordered pass,
+    # and its fallback when a list would overflow (every score equal puts every key
+    # in one bin; k above the space for the keys above the cut bin)
+    w = synth.scaled(W["gqa_32k"], max_ctx=50000, batch=1, num_q_heads=8, num_kv_heads=2)
+    if case == "k_above_list_space":
+        w = w.replace(topk_num=0, topk_den=0, topk_abs=9000)
+    cpu = synth.make_inputs(w)
+    if case == "equal_scores":
+        cpu["q"].zero_()
     check(w, inputs=cpu)
 
 
@@ -211,6 +225,29 @@ def test_bad_length_sets_error():
     got, err = run_gpu(w, _to(cpu, dev))
     assert err & _abi.VATTN_DEV_BAD_SEQLEN
     assert np.all(got["out"] == 0)
+
+
+def test_context_reuse_with_fewer_items_than_record_producers():
+    # one context, two calls: the first gathers more items than the gathers have
+    # record producers (every producer writes records), the second fewer (most
+    # producers own no item and write no record), so the second call must read
+    # only the records it wrote, not the first call's left in the workspace
+    w = SMALL["tiny_f32"]
+    dev = _cuda()
+    cpu = synth.make_inputs(w)
+    x = _to(cpu, dev)
+    dec = decoder_for(w)
+    try:
+        for topk in (1500, w.topk_abs):
+            wc = w.replace(topk_abs=topk)
+            res = dec.decode(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["seq_lens"],
+                             params_for(wc, x))
+            torch.cuda.synchronize()
+            assert dec.last_error() == 0
+            got = {k: v.cpu().numpy() for k, v in res.items()}
+            compare(wc, got, oracle.decode(oracle.make_problem(wc), cpu), range(w.units))
+    finally:
+        dec.close()
 
 
 def test_bounded_wait_runs_out_and_reports_a_timeout():

@@ -91,8 +91,8 @@ def test_edge_lengths_paged():
     check(w, inputs=cpu)
 
 
-def test_long_context_cluster_select():
-    # a middle longer than one CTA's staging takes the cluster select after k_topp
+def test_long_context_streamed_select():
+    # a middle longer than one CTA's shared memory takes the streamed select after k_topp
     check(_p(synth.scaled(W["gqa_32k"], max_ctx=50000, batch=1, num_q_heads=8, num_kv_heads=2), 4, 5))
 
 

@@ -20,7 +20,6 @@ struct vattn_ctx {
   int num_sms = 0;
   int G = 1;
   int units_max = 0;
-  int nseg = 0;
   int score_grid = 0;
   bool score_tma = false;   // contiguous cache: the bulk-copy score pass
   size_t score_smem = 0;
@@ -28,8 +27,7 @@ struct vattn_ctx {
   int CD = 0, CS = 0;      // record producers (warps) of the det/dense and sample gathers
   size_t gather_smem = 0;   // gathers (all modes)
   int gather_threads = 0;
-  bool select1 = false;     // one CTA per unit selects the top-k and draws the pilot
-  size_t select_smem = 0;   // else one cluster per unit (0: four grid-wide passes)
+  bool select1 = false;     // k_select1 (keys staged in shared memory), else k_topk
   int draw_splits = 1;
   size_t ws_bytes = 0;
   void* ws = nullptr;
@@ -40,7 +38,6 @@ struct vattn_ctx {
   int* dims = nullptr;
   unsigned* ordk = nullptr;
   unsigned* hist = nullptr;
-  unsigned* segcnt = nullptr;
   float* pscore = nullptr;
   int* num_need = nullptr;
   long long* prefix = nullptr;
@@ -135,6 +132,9 @@ struct Kernels {
   void (*det)(DevParams);
   void (*sample)(DevParams);
   void (*dense)(DevParams);
+  void (*det_host)(DevParams);     // the gathers for caches in host memory
+  void (*sample_host)(DevParams);
+  void (*dense_host)(DevParams);
   void (*budget)(DevParams);
   void (*numstats)(DevParams);
   void (*combine_sample)(DevParams);
@@ -157,6 +157,9 @@ Kernels kernels_for() {
   k.det = vattn::k_gather<T, D, G, vattn::kModeDet>;
   k.sample = vattn::k_gather<T, D, G, vattn::kModeSample>;
   k.dense = vattn::k_gather<T, D, G, vattn::kModeDense>;
+  k.det_host = vattn::k_gather<T, D, G, vattn::kModeDet, true>;
+  k.sample_host = vattn::k_gather<T, D, G, vattn::kModeSample, true>;
+  k.dense_host = vattn::k_gather<T, D, G, vattn::kModeDense, true>;
   k.budget = vattn::k_budget<D, G>;
   k.numstats = vattn::k_numstats<T, D, G>;
   k.combine_sample = vattn::k_combine<D, G, vattn::kModeSample>;
@@ -251,18 +254,14 @@ void fill_common(const vattn_ctx* ctx, DevParams* P, int batch) {
   P->rank = c.proxy_rank;
   P->kv_host = c.kv_location == VATTN_KV_HOST;
   P->scale = static_cast<float>(1.0 / sqrt(static_cast<double>(c.head_dim)));
-  P->nseg = ctx->nseg;
   P->info = ctx->info;
   P->qbar = ctx->qbar;
   P->qsel = ctx->qsel;
   P->dims = ctx->dims;
   P->ordk = ctx->ordk;
   P->hist = ctx->hist;
-  P->segcnt = ctx->segcnt;
   P->pscore = ctx->pscore;
   P->num_need = ctx->num_need;
-  // only the grid-wide select reads the digit-2 and digit-3 histograms
-  P->hist_words = (ctx->select1 || ctx->select_smem) ? vattn::kHist1 : vattn::kHistAll;
   P->prefix = ctx->prefix;
   P->gcnt = ctx->gcnt;
   P->pre_det = ctx->pre_det;
@@ -291,6 +290,15 @@ void launch(void (*kern)(DevParams), dim3 grid, dim3 block, size_t smem, cudaStr
   cfg.numAttrs = 1;
   cudaLaunchKernelEx(&cfg, kern, P);
   (*count)++;
+}
+
+// Threads of a combine CTA (one per unit and head): eight record groups per
+// dimension while the CTAs fit one wave at two per SM, else two (a wave of
+// 256-thread CTAs).
+int comb_threads(const vattn_ctx* ctx, int units) {
+  const long long ctas = static_cast<long long>(units) * ctx->G;
+  const int groups = ctas <= 2LL * ctx->num_sms ? vattn::kCombGroups : 2;
+  return groups * ctx->cfg.head_dim;
 }
 
 int finish(vattn_ctx* ctx, int launches) {
@@ -335,7 +343,6 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const int D = cfg->head_dim, G = ctx->G;
   const size_t U = static_cast<size_t>(cfg->max_batch) * cfg->num_kv_heads;
   ctx->units_max = static_cast<int>(U);
-  ctx->nseg = (cfg->max_ctx + vattn::kSeg - 1) / vattn::kSeg;
 
   // grid sizes: the score pass and the gathers run one wave of resident CTAs
   void (*score)(DevParams) = cfg->proxy == VATTN_SPARQ ? K.score_sparq
@@ -358,7 +365,7 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   }
   ctx->gather_smem = K.gather_smem;
   ctx->gather_threads = K.gather_threads;
-  for (auto fn : {K.det, K.sample, K.dense})
+  for (auto fn : {K.det, K.sample, K.dense, K.det_host, K.sample_host, K.dense_host})
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->gather_smem));
   cudaFuncSetAttribute(K.numstats, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(vattn::kNumSmem));
   int gocc = 0;
@@ -376,8 +383,7 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const size_t sz_info = align256(U * sizeof(UnitInfo));
   const size_t sz_vec = align256(U * D * sizeof(float));
   const size_t sz_ordk = align256(U * cfg->max_ctx * sizeof(unsigned));
-  const size_t sz_hist = align256(U * vattn::kHistAll * sizeof(unsigned));
-  const size_t sz_seg = align256(U * ctx->nseg * 2 * sizeof(unsigned));
+  const size_t sz_hist = align256(U * vattn::kHist1 * sizeof(unsigned));
   const size_t sz_ps = align256(U * cfg->max_ctx * G * sizeof(float));
   const size_t sz_nneed = align256(U * G * sizeof(int));
   const size_t sz_pre = align256((U + 1) * sizeof(long long));
@@ -386,7 +392,7 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   const size_t sz_rdet = align256((ctx->CD + 2 * U) * REC * sizeof(float));
   const size_t sz_rsmp = align256((ctx->CS + 2 * U) * REC * sizeof(float));
   const size_t sz_err = 256;
-  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_seg + sz_ps + sz_nneed + sz_pre + sz_gcnt +
+  ctx->ws_bytes = sz_info + 3 * sz_vec + sz_ordk + sz_hist + sz_ps + sz_nneed + sz_pre + sz_gcnt +
                   2 * sz_spre + sz_rdet + sz_rsmp + sz_err;
   if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -400,7 +406,6 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->dims = reinterpret_cast<int*>(p); p += sz_vec;
   ctx->ordk = reinterpret_cast<unsigned*>(p); p += sz_ordk;
   ctx->hist = reinterpret_cast<unsigned*>(p); p += sz_hist;
-  ctx->segcnt = reinterpret_cast<unsigned*>(p); p += sz_seg;
   ctx->pscore = reinterpret_cast<float*>(p); p += sz_ps;
   ctx->num_need = reinterpret_cast<int*>(p); p += sz_nneed;
   ctx->prefix = reinterpret_cast<long long*>(p); p += sz_pre;
@@ -415,23 +420,18 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
     delete ctx;
     return VATTN_ECUDA;
   }
-  // the top-k selection: one CTA per unit when the middle's keys fit in its
-  // shared memory, else one cluster per unit when each CTA's segment fits,
-  // else four grid-wide passes
+  // the top-k selection: one CTA per unit with the middle's keys staged in
+  // its shared memory when they fit, else one CTA per unit streaming them
   ctx->select1 = cfg->max_ctx <= vattn::kSel1MaxKeys &&
                  cudaFuncSetAttribute(vattn::k_select1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(vattn::kSel1Smem)) == cudaSuccess;
   cudaGetLastError();
-  {
-    const size_t seg = (static_cast<size_t>(cfg->max_ctx) + vattn::kSelCluster - 1) / vattn::kSelCluster;
-    const size_t bytes = vattn::kSelFixedSmem + seg * sizeof(unsigned);
-    int optin = 0;
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device);
-    if (bytes + 1024 <= static_cast<size_t>(optin) &&
-        cudaFuncSetAttribute(vattn::k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bytes)) == cudaSuccess)
-      ctx->select_smem = bytes;
-    cudaGetLastError();
+  if (!ctx->select1 &&
+      cudaFuncSetAttribute(vattn::k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess) {
+    cudaFree(ctx->ws);
+    delete ctx;
+    return VATTN_ECUDA;
   }
   *out = ctx;
   return VATTN_OK;
@@ -564,7 +564,6 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   P.budgets = budgets;
   P.head_need = head_need;
   P.dense = 0;
-  const dim3 seg_grid(P.units, ctx->nseg);
 
   int launches = 0;
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
@@ -592,27 +591,20 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   }
   // top-p: each unit's top-k size from the mass of its ranking scores
   if (P.topp_den > 0) launch(vattn::k_topp, dim3(P.units), dim3(vattn::kToppThreads), 0, st, P, &launches);
-  if (ctx->select1) {
+  // top-k select and pilot draws: keys staged in one CTA's shared memory when
+  // the middle fits, else streamed from L2 by k_topk
+  if (ctx->select1)
     launch(vattn::k_select1, dim3(P.units), dim3(vattn::kSel1Threads), vattn::kSel1Smem, st, P, &launches);
-  } else {
-    if (ctx->select_smem) {
-      launch(vattn::k_select, dim3(P.units * vattn::kSelCluster), dim3(256), ctx->select_smem, st, P, &launches);
-    } else {
-      launch(vattn::k_sel_hist<2>, seg_grid, dim3(256), 0, st, P, &launches);
-      launch(vattn::k_sel_hist<3>, seg_grid, dim3(256), 0, st, P, &launches);
-      launch(vattn::k_sel_count, seg_grid, dim3(256), 0, st, P, &launches);
-      launch(vattn::k_sel_write, seg_grid, dim3(256), 0, st, P, &launches);
-    }
-    launch(vattn::k_draws<0>, dim3(P.units, ctx->draw_splits), dim3(128), 0, st, P, &launches);
-  }
-  launch(K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  else
+    launch(vattn::k_topk, dim3(P.units), dim3(vattn::kTopkThreads), vattn::kTopkKernelSmem, st, P, &launches);
+  launch(P.kv_host ? K.det_host : K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   if (P.guarantee)
     launch(K.numstats, dim3(P.units, (ctx->G * c.head_dim + vattn::kNumThreads - 1) / vattn::kNumThreads),
            dim3(vattn::kNumThreads), vattn::kNumSmem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(vattn::kBudgetThreads), 0, st, P, &launches);
-  launch(vattn::k_draws<1>, dim3(P.units, ctx->draw_splits * 4), dim3(128), 0, st, P, &launches);
-  launch(K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
-  launch(K.combine_sample, dim3(P.units, ctx->G), dim3(vattn::kCombGroups * c.head_dim), 0, st, P, &launches);
+  launch(vattn::k_draws, dim3(P.units, ctx->draw_splits * 4), dim3(128), 0, st, P, &launches);
+  launch(P.kv_host ? K.sample_host : K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  launch(K.combine_sample, dim3(P.units, ctx->G), dim3(comb_threads(ctx, P.units)), 0, st, P, &launches);
   return finish(ctx, launches);
 }
 
@@ -657,8 +649,8 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.sel = reinterpret_cast<int*>(ctx->ordk);
   int launches = 0;
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
-  launch(K.dense, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
-  launch(K.combine_dense, dim3(P.units, ctx->G), dim3(vattn::kCombGroups * c.head_dim), 0, st, P, &launches);
+  launch(P.kv_host ? K.dense_host : K.dense, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  launch(K.combine_dense, dim3(P.units, ctx->G), dim3(comb_threads(ctx, P.units)), 0, st, P, &launches);
   return finish(ctx, launches);
 }
 

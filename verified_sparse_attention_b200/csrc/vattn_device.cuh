@@ -22,8 +22,6 @@ constexpr unsigned kDevTimeout = 4u;
 constexpr int kHist1 = 2048;  // bins of digit 1 (key bits 31..21)
 constexpr int kHist2 = 2048;  // bins of digit 2 (key bits 20..10)
 constexpr int kHist3 = 1024;  // bins of digit 3 (key bits 9..0)
-constexpr int kHistAll = kHist1 + kHist2 + kHist3;
-constexpr int kSeg = 4096;         // positions per selection CTA (256 threads x 16)
 constexpr int kTopkSmem = 6144;    // top-k lists up to this length are staged in shared memory
 
 // Per-unit (sequence b, KV head h) state written by the prep and budget kernels.
@@ -61,7 +59,7 @@ struct DevParams {
   float eps, scale;
   double z;
   unsigned long long seed;
-  int nseg, dense;
+  int dense;
   int guarantee;    // 1: the budget also bounds the numerator vector (output guarantee)
   int topp_num, topp_den;  // topp_den > 0: top-p selection with p = topp_num / topp_den
   int kv_host;      // 1: k and v point into mapped host memory (plain loads only)
@@ -88,11 +86,9 @@ struct DevParams {
   float* qsel;      // [units][D]: SparQ query values at the chosen dims, or the Loki projected query
   int* dims;        // [units][D]: SparQ chosen dims, ascending
   unsigned* ordk;   // [units][max_ctx]: ranking-score keys over the middle
-  unsigned* hist;   // [units][kHistAll]
-  unsigned* segcnt; // [units][nseg][2]
+  unsigned* hist;   // [units][kHist1]: digit-1 histogram of the ranking keys
   float* pscore;    // [units][max_ctx][G]: true scores of I_f and the pilot
   int* num_need;    // [units][G]: numerator sizes n_v (output guarantee)
-  int hist_words;   // histogram words per unit that k_prep zeroes (all only for the grid-wide select)
   long long* prefix;// [units + 1]: score-pass work prefix
   unsigned* gcnt;   // [0]: score-pass chunks handed out, [1]: units done by k_topp (zeroed by k_prep)
   long long* pre_det;   // [2 units + 1]: slice prefix of the det (or dense) gather

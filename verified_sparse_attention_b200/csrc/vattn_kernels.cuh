@@ -1,21 +1,25 @@
 // Kernels of one verified-sparse-attention decode step, in launch order:
 //
 //   k_prep        per unit: validate, regions, ranking query, proxy query,
-//                 zero the radix histograms, write sinks/window indices; one
-//                 extra CTA writes the score-pass work prefix over units
-//   k_score_rows  exact (q.k) or Loki (projected q . projected k) ranking
-//                 scores over the middle region, streamed from HBM; writes
-//                 order keys and the first radix digit's histogram
-//   k_score_sparq SparQ proxy scores from the dim-major K copy
-//   k_sel_hist    radix-select digits 2 and 3 (key bits 20..10, 9..0)
-//   k_sel_count   exact threshold; counts above / equal per segment
-//   k_sel_write   ordered compaction of the top-k positions (ascending)
+//                 zero the digit-1 histogram, write sinks/window indices; one
+//                 extra CTA writes the score-pass work prefix and the det
+//                 gather's slice prefix
+//   k_score_tma   exact or Loki ranking scores of a contiguous cache, streamed
+//   k_score_rows  through bulk copies (k_score_rows: paged caches, or caches
+//   k_score_sparq in host memory; k_score_sparq: the SparQ proxy from the
+//                 dim-major K copy); writes the order keys and the histogram
+//                 of their first radix digit
+//   k_topp        (top-p only) each unit's top-k size from its scores' mass
+//   k_select1     top-k select and pilot draws, one CTA per unit, keys staged
+//   k_topk        in shared memory (k_topk: any middle length, keys streamed)
 //   k_gather<det>    gather + softmax-accumulate of I_f and the pilot draws
-//                    (true scores of every query head kept); the unit's last
-//                    CTA computes the per-head CLT budgets
-//   k_gather<sample> the remaining draws (or the whole tail); the unit's last
-//                    CTA merges its records, reweights the sample by N_tail / b
-//                    and writes out (k_gather<dense>: all positions)
+//                    (true scores of every query head kept)
+//   k_numstats    (output guarantee only) numerator statistics of the pilot
+//   k_budget      per-head CLT budgets from the pilot statistics
+//   k_draws       the rest of the sample's positions; the sample slice prefix
+//   k_gather<sample> the remaining draws (or the whole tail)
+//   k_combine<sample> merge the records, reweight the sample by N_tail / b,
+//                    write out (k_gather<dense> + k_combine<dense>: dense decode)
 //
 // A unit is one (sequence b, KV head h); u = b * Hkv + h. The method follows
 // "vAttention: A New Approach to Sparse Attention with Guaranteed Accuracy",
@@ -86,6 +90,8 @@ __device__ __forceinline__ void grid_dependents_launch() {
 }
 
 // ============================================================ k_prep
+constexpr int kPrepLens = 1024;  // sequence lengths the prefix CTA keeps in shared memory
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   __shared__ float s_q[D];
@@ -97,17 +103,26 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   grid_dependency_wait();  // the previous call's kernels still read this workspace
 
   if (u == P.units) {
+    // the validated lengths once into shared memory (the scans below then run
+    // without a global load per round)
+    __shared__ int s_len[kPrepLens];
+    auto seq_len = [&](int bq) -> int {
+      int n = bq < kPrepLens ? s_len[bq] : P.seq_lens[bq];
+      if (bq >= kPrepLens && (n < 0 || n > P.max_ctx)) n = 0;
+      return n;
+    };
+    for (int i = tid; i < min(P.batch, kPrepLens); i += blockDim.x) {
+      const int n = P.seq_lens[i];
+      s_len[i] = (n < 0 || n > P.max_ctx) ? 0 : n;
+    }
+    __syncthreads();
     // work prefix over units for the persistent score pass
     constexpr int V = Elem<T>::kPer16;
     long long carry = 0;
     for (int base = 0; base < P.units; base += blockDim.x) {
       const int uu = base + tid;
       long long w = 0;
-      if (uu < P.units) {
-        int n = P.seq_lens[uu / P.Hkv];
-        if (n < 0 || n > P.max_ctx) n = 0;
-        w = score_work(P, n, V);
-      }
+      if (uu < P.units) w = score_work(P, seq_len(uu / P.Hkv), V);
       // work per unit <= max_ctx <= 2^24, so a 128-unit chunk sum fits in 32 bits
       const unsigned incl = block_inclusive_scan(static_cast<unsigned>(w), s_warp);
       if (uu < P.units) P.prefix[uu] = carry + (incl - static_cast<unsigned>(w));
@@ -126,8 +141,7 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
       const int sidx = base + tid;
       unsigned cnt = 0;
       if (sidx < ns) {
-        int n = P.seq_lens[(sidx >> 1) / P.Hkv];
-        if (n < 0 || n > P.max_ctx) n = 0;
+        const int n = seq_len((sidx >> 1) / P.Hkv);
         if (P.dense) {
           cnt = (sidx & 1) ? 0u : static_cast<unsigned>(n);
         } else {
@@ -161,9 +175,16 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   if (bad_len) n = 0;
   const int npages = (n + P.ps - 1) / P.ps;
   int bad = 0;
-  for (int i = tid; i < npages; i += blockDim.x) {
-    const int pid = P.page_table[static_cast<size_t>(b) * P.pps + i];
-    if (pid < 0 || pid >= P.num_pages) bad = 1;
+  for (int i0 = tid; i0 < npages; i0 += 8 * blockDim.x) {  // eight independent loads in flight
+    int pid[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      const int i = i0 + j * blockDim.x;
+      pid[j] = i < npages ? P.page_table[static_cast<size_t>(b) * P.pps + i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+      if (pid[j] < 0 || pid[j] >= P.num_pages) bad = 1;
   }
   bad = __syncthreads_or(bad);
   if (tid == 0 && h == 0) {
@@ -234,15 +255,21 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
   } else if (P.proxy == kProxyLoki) {
     // projected ranking query: one fused chain over d per component
     if (tid < P.rank) {
+      // the basis column's loads go out sixteen at a time; the chain stays in order
       float acc = 0.0f;
-      for (int i = 0; i < D; i++)
-        acc = __fmaf_rn(s_q[i], P.basis[(static_cast<size_t>(h) * D + i) * P.rank + tid], acc);
+      for (int i0 = 0; i0 < D; i0 += 16) {
+        float bv[16];
+#pragma unroll
+        for (int j = 0; j < 16; j++) bv[j] = P.basis[(static_cast<size_t>(h) * D + i0 + j) * P.rank + tid];
+#pragma unroll
+        for (int j = 0; j < 16; j++) acc = __fmaf_rn(s_q[i0 + j], bv[j], acc);
+      }
       P.qsel[static_cast<size_t>(u) * D + tid] = acc;
     }
   }
 
-  unsigned* hist = P.hist + static_cast<size_t>(u) * kHistAll;
-  for (int i = tid; i < P.hist_words; i += blockDim.x) hist[i] = 0u;
+  unsigned* hist = P.hist + static_cast<size_t>(u) * kHist1;
+  for (int i = tid; i < kHist1; i += blockDim.x) hist[i] = 0u;
   int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
   for (int i = tid; i < r.s1; i += blockDim.x) sel[i] = i;
   if (P.topp_den == 0)  // with top-p, k_topp writes the window once k is known
@@ -350,7 +377,7 @@ __global__ void __launch_bounds__(256) k_score_rows(DevParams P) {
           atomicAdd(&s_hist[o >> 21], 1u);
         }
       }
-      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
+      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHist1);
     }
     cur = uend;
   }
@@ -447,360 +474,10 @@ __global__ void __launch_bounds__(256) k_score_sparq(DevParams P) {
           }
         }
       }
-      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
+      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHist1);
     }
     cur = uend;
   }
-}
-
-// ============================================================ radix select
-// Digits resolved so far for unit u, recomputed by each CTA from the global
-// histograms (cheap: three block scans).
-struct SelState {
-  int d1, d2, d3, krem;
-};
-
-template <int DEPTH>
-__device__ __forceinline__ SelState resolve_digits(const DevParams& P, int u, int k) {
-  __shared__ int s_digit, s_krem;
-  __shared__ unsigned s_warp[32];
-  const unsigned* hist = P.hist + static_cast<size_t>(u) * kHistAll;
-  SelState st{0, 0, 0, k};
-  if (threadIdx.x == 0) { s_digit = 0; s_krem = k; }
-  __syncthreads();
-  find_digit<kHist1>(hist, st.krem, &s_digit, &s_krem, s_warp);
-  st.d1 = s_digit;
-  st.krem = s_krem;
-  __syncthreads();
-  if (DEPTH >= 2) {
-    find_digit<kHist2>(hist + kHist1, st.krem, &s_digit, &s_krem, s_warp);
-    st.d2 = s_digit;
-    st.krem = s_krem;
-    __syncthreads();
-  }
-  if (DEPTH >= 3) {
-    find_digit<kHist3>(hist + kHist1 + kHist2, st.krem, &s_digit, &s_krem, s_warp);
-    st.d3 = s_digit;
-    st.krem = s_krem;
-    __syncthreads();
-  }
-  return st;
-}
-
-// Histogram of digit PASS (2 or 3) over keys matching the digits above it.
-template <int PASS>
-__global__ void __launch_bounds__(256) k_sel_hist(DevParams P) {
-  __shared__ unsigned s_h[kHist2];
-  const int u = blockIdx.x, seg = blockIdx.y;
-  grid_dependency_wait();
-  const UnitInfo inf = P.info[u];
-  if (inf.k <= 0) return;
-  const int pb = inf.s1 + seg * kSeg;
-  const int pe = min(inf.wst, pb + kSeg);
-  if (pb >= pe) return;
-  const SelState st = resolve_digits<PASS - 1>(P, u, inf.k);
-  constexpr int NB = PASS == 2 ? kHist2 : kHist3;
-  for (int i = threadIdx.x; i < NB; i += blockDim.x) s_h[i] = 0u;
-  __syncthreads();
-  const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
-  const unsigned pre = PASS == 2 ? static_cast<unsigned>(st.d1)
-                                 : (static_cast<unsigned>(st.d1) << 11 | static_cast<unsigned>(st.d2));
-  constexpr int PER = kSeg / 256;
-  unsigned keys[PER];
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = pb + threadIdx.x + 256 * i;
-    keys[i] = j < pe ? ordk[j] : 0u;
-  }
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = pb + threadIdx.x + 256 * i;
-    const unsigned o = keys[i];
-    if (j >= pe) continue;
-    if (PASS == 2) {
-      if ((o >> 21) == pre) atomicAdd(&s_h[(o >> 10) & 2047u], 1u);
-    } else {
-      if ((o >> 10) == pre) atomicAdd(&s_h[o & 1023u], 1u);
-    }
-  }
-  __syncthreads();
-  unsigned* g = P.hist + static_cast<size_t>(u) * kHistAll + (PASS == 2 ? kHist1 : kHist1 + kHist2);
-  for (int i = threadIdx.x; i < NB; i += blockDim.x)
-    if (s_h[i]) atomicAdd(g + i, s_h[i]);
-}
-
-// Threshold key thr (the k-th largest) and need_eq (keys equal to thr to take,
-// lowest positions first); counts of keys above / equal to thr per segment.
-__global__ void __launch_bounds__(256) k_sel_count(DevParams P) {
-  __shared__ unsigned s_warp[32];
-  const int u = blockIdx.x, seg = blockIdx.y;
-  grid_dependency_wait();
-  const UnitInfo inf = P.info[u];
-  if (inf.k <= 0) return;
-  const int pb = inf.s1 + seg * kSeg;
-  const int pe = min(inf.wst, pb + kSeg);
-  if (pb >= pe) return;
-  const SelState st = resolve_digits<3>(P, u, inf.k);
-  const unsigned thr = static_cast<unsigned>(st.d1) << 21 | static_cast<unsigned>(st.d2) << 10 |
-                       static_cast<unsigned>(st.d3);
-  const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
-  unsigned gt = 0, eq = 0;
-  constexpr int PER = kSeg / 256;
-  unsigned keys[PER];
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = pb + threadIdx.x + 256 * i;
-    keys[i] = j < pe ? ordk[j] : 0u;
-  }
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = pb + threadIdx.x + 256 * i;
-    if (j < pe) {
-      gt += keys[i] > thr;
-      eq += keys[i] == thr;
-    }
-  }
-  gt = block_sum(gt, s_warp);
-  eq = block_sum(eq, s_warp);
-  if (threadIdx.x == 0) {
-    unsigned* c = P.segcnt + (static_cast<size_t>(u) * P.nseg + seg) * 2;
-    c[0] = gt;
-    c[1] = eq;
-    if (seg == 0) {
-      P.info[u].thr = thr;
-      P.info[u].need_eq = st.krem;
-    }
-  }
-}
-
-// Ordered compaction: each CTA writes the selected positions of its segment
-// at their final ascending rank in sel_idx[s1 ...].
-__global__ void __launch_bounds__(256) k_sel_write(DevParams P) {
-  __shared__ unsigned s_warp[32];
-  __shared__ unsigned s_before[2];
-  const int u = blockIdx.x, seg = blockIdx.y;
-  grid_dependency_wait();
-  const UnitInfo inf = P.info[u];
-  if (inf.k <= 0) return;
-  const int pb = inf.s1 + seg * kSeg;
-  const int pe = min(inf.wst, pb + kSeg);
-  if (pb >= pe) return;
-  const unsigned thr = inf.thr;
-  const unsigned need_eq = static_cast<unsigned>(inf.need_eq);
-  if (threadIdx.x < 2) {
-    unsigned acc = 0;
-    for (int s = 0; s < seg; s++) acc += P.segcnt[(static_cast<size_t>(u) * P.nseg + s) * 2 + threadIdx.x];
-    s_before[threadIdx.x] = acc;
-  }
-  __syncthreads();
-  const unsigned gt_before = s_before[0], eq_before = s_before[1];
-  const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
-  constexpr int PER = kSeg / 256;
-  const int j0 = pb + threadIdx.x * PER;
-  unsigned keys[PER];
-  unsigned neq = 0;
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = j0 + i;
-    keys[i] = j < pe ? ordk[j] : 0u;
-    neq += (j < pe) && keys[i] == thr;
-  }
-  const unsigned eq_incl = block_inclusive_scan(neq, s_warp);
-  unsigned eq_rank = eq_before + eq_incl - neq;
-  bool take[PER];
-  unsigned ntake = 0;
-#pragma unroll
-  for (int i = 0; i < PER; i++) {
-    const int j = j0 + i;
-    const bool valid = j < pe;
-    const bool e = valid && keys[i] == thr;
-    take[i] = valid && (keys[i] > thr || (e && eq_rank < need_eq));
-    eq_rank += e;
-    ntake += take[i];
-  }
-  const unsigned take_incl = block_inclusive_scan(ntake, s_warp);
-  unsigned pos = gt_before + min(eq_before, need_eq) + take_incl - ntake;
-  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
-#pragma unroll
-  for (int i = 0; i < PER; i++)
-    if (take[i]) sel[pos++] = j0 + i;
-}
-
-// ============================================================ k_select (cluster)
-// The whole top-k selection of one unit in one cluster of kSelCluster CTAs.
-// CTA r of the cluster owns a contiguous segment of the middle's keys, staged
-// once in its shared memory. Digits 2 and 3 of the radix select are found
-// from cluster-wide histograms: every CTA histograms its segment, CTA r sums
-// bin slice r over the cluster (distributed shared memory), and every CTA
-// gathers the summed slices. The counts above / equal to the threshold are
-// exchanged the same way, and each CTA compacts its segment in order. Phases
-// are separated by cluster barriers.
-constexpr int kSelCluster = 8;
-constexpr int kSelFixedSmem = (kHist2 + kHist2 / kSelCluster + kHist2) * 4 + 64;
-
-__device__ __forceinline__ unsigned* cluster_peer(unsigned* p, int rank) {
-  return cooperative_groups::this_cluster().map_shared_rank(p, rank);
-}
-
-// Cluster-wide histogram of NB bins from each CTA's s_loc; result in s_full.
-template <int NB>
-__device__ __forceinline__ void cluster_hist_allreduce(unsigned* s_loc, unsigned* s_red, unsigned* s_full,
-                                                       int rank) {
-  auto cluster = cooperative_groups::this_cluster();
-  constexpr int SL = NB / kSelCluster;  // bins summed by each CTA
-  cluster.sync();
-  for (int x = threadIdx.x; x < SL; x += blockDim.x) {
-    unsigned acc = 0;
-#pragma unroll
-    for (int q = 0; q < kSelCluster; q++) acc += cluster_peer(s_loc, q)[rank * SL + x];
-    s_red[x] = acc;
-  }
-  cluster.sync();
-  for (int x = threadIdx.x; x < NB; x += blockDim.x) s_full[x] = cluster_peer(s_red, x / SL)[x % SL];
-  cluster.sync();  // s_red and s_loc may be reused after every CTA gathered
-}
-
-__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(256) k_select(DevParams P) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned* s_loc = reinterpret_cast<unsigned*>(smem);  // [kHist2] local histogram
-  unsigned* s_red = s_loc + kHist2;                      // [kHist2 / cluster] summed slice
-  unsigned* s_full = s_red + kHist2 / kSelCluster;       // [kHist2] cluster histogram
-  unsigned* s_cnt = s_full + kHist2;                     // [2] this CTA's counts above / equal
-  unsigned* s_keys = reinterpret_cast<unsigned*>(smem + kSelFixedSmem);
-  __shared__ unsigned s_warp[32];
-  __shared__ int s_digit, s_krem;
-  auto cluster = cooperative_groups::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int u = blockIdx.x / kSelCluster;
-  grid_dependency_wait();
-  const UnitInfo inf = P.info[u];
-  if (inf.k <= 0) return;  // uniform over the cluster: no peer touches this CTA
-  const int mlen = inf.wst - inf.s1;
-  const int seglen = (mlen + kSelCluster - 1) / kSelCluster;
-  const int pb = inf.s1 + rank * seglen;
-  const int pe = min(inf.wst, pb + seglen);
-  const int cnt = max(0, pe - pb);
-  const unsigned* ordk = P.ordk + static_cast<size_t>(u) * P.max_ctx;
-  for (int base = 0; base < cnt; base += 16 * 256) {  // 16 independent loads in flight per thread
-    unsigned v[16];
-#pragma unroll
-    for (int i = 0; i < 16; i++) {
-      const int x = base + i * 256 + threadIdx.x;
-      v[i] = x < cnt ? ordk[pb + x] : 0u;
-    }
-#pragma unroll
-    for (int i = 0; i < 16; i++) {
-      const int x = base + i * 256 + threadIdx.x;
-      if (x < cnt) s_keys[x] = v[i];
-    }
-  }
-  __syncthreads();
-
-  // digit 1 from the score pass's histogram (every CTA resolves it)
-  if (threadIdx.x == 0) {
-    s_digit = 0;
-    s_krem = inf.k;
-  }
-  __syncthreads();
-  const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHistAll;
-  find_digit<kHist1>(h1, inf.k, &s_digit, &s_krem, s_warp);
-  const unsigned d1 = static_cast<unsigned>(s_digit);
-  const int krem1 = s_krem;
-
-  // digit 2
-  for (int x = threadIdx.x; x < kHist2; x += blockDim.x) s_loc[x] = 0u;
-  __syncthreads();
-  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
-    const unsigned o = s_keys[x];
-    if ((o >> 21) == d1) atomicAdd(&s_loc[(o >> 10) & 2047u], 1u);
-  }
-  cluster_hist_allreduce<kHist2>(s_loc, s_red, s_full, rank);
-  find_digit<kHist2>(s_full, krem1, &s_digit, &s_krem, s_warp);
-  const unsigned d2 = static_cast<unsigned>(s_digit);
-  const int krem2 = s_krem;
-
-  // digit 3
-  const unsigned pre = d1 << 11 | d2;
-  for (int x = threadIdx.x; x < kHist3; x += blockDim.x) s_loc[x] = 0u;
-  __syncthreads();
-  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
-    const unsigned o = s_keys[x];
-    if ((o >> 10) == pre) atomicAdd(&s_loc[o & 1023u], 1u);
-  }
-  cluster_hist_allreduce<kHist3>(s_loc, s_red, s_full, rank);
-  find_digit<kHist3>(s_full, krem2, &s_digit, &s_krem, s_warp);
-  const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
-  const unsigned need_eq = static_cast<unsigned>(s_krem);
-
-  // counts above / equal per CTA, exchanged over the cluster
-  unsigned gt = 0, eq = 0;
-  for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
-    const unsigned o = s_keys[x];
-    gt += o > thr;
-    eq += o == thr;
-  }
-  gt = block_sum(gt, s_warp);
-  eq = block_sum(eq, s_warp);
-  if (threadIdx.x == 0) {
-    s_cnt[0] = gt;
-    s_cnt[1] = eq;
-  }
-  cluster.sync();
-  unsigned gt_before = 0, eq_before = 0;
-  for (int q = 0; q < rank; q++) {
-    const unsigned* pc = cluster_peer(s_cnt, q);
-    gt_before += pc[0];
-    eq_before += pc[1];
-  }
-  if (rank == 0 && threadIdx.x == 0) {
-    P.info[u].thr = thr;
-    P.info[u].need_eq = static_cast<int>(need_eq);
-  }
-
-  // ordered compaction of the segment, 16 consecutive keys per thread per round
-  int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
-  unsigned taken = gt_before + min(eq_before, need_eq);
-  unsigned eq_seen = eq_before;
-  constexpr int PER = 16;
-  for (int base = 0; base < cnt; base += PER * 256) {
-    const int x0 = base + threadIdx.x * PER;
-    unsigned neq = 0;
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      const int x = x0 + i;
-      neq += (x < cnt) && s_keys[x] == thr;
-    }
-    const unsigned eq_incl = block_inclusive_scan(neq, s_warp);
-    unsigned eq_rank = eq_seen + eq_incl - neq;
-    unsigned tk = 0;
-    bool take[PER];
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      const int x = x0 + i;
-      const bool valid = x < cnt;
-      const unsigned o = valid ? s_keys[x] : 0u;
-      const bool e = valid && o == thr;
-      take[i] = valid && (o > thr || (e && eq_rank < need_eq));
-      eq_rank += e;
-      tk += take[i];
-    }
-    const unsigned tk_incl = block_inclusive_scan(tk, s_warp);
-    unsigned pos = taken + tk_incl - tk;
-#pragma unroll
-    for (int i = 0; i < PER; i++)
-      if (take[i]) sel[pos++] = pb + x0 + i;
-    // totals of this round for the next one (last thread holds the inclusive sums)
-    __shared__ unsigned s_round[2];
-    if (threadIdx.x == blockDim.x - 1) {
-      s_round[0] = eq_incl;
-      s_round[1] = tk_incl;
-    }
-    __syncthreads();
-    eq_seen += s_round[0];
-    taken += s_round[1];
-    __syncthreads();
-  }
-  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
 // ============================================================ tail positions
@@ -1024,16 +701,31 @@ __device__ void write_slice_prefix(const DevParams& P, long long* pre, unsigned*
   if (threadIdx.x == 0) pre[ns] = *s_carry;
 }
 
-// Records of slice s: CTAs [c_first, c_last] (empty when c_first > c_last).
-__device__ __forceinline__ void slice_ctas(const long long* pre, int s, long long T, int C, int& cf,
-                                           int& cl) {
-  if (pre[s + 1] <= pre[s]) {
-    cf = 1;
-    cl = 0;
-    return;
+// The records of slice s: one from every producer that owns at least one of
+// its items (a producer that owns no item writes none). With T >= C every
+// producer owns items, so they are the producers [c_first, c_last]; with
+// T < C each owns at most one, so they are the owners of the slice's items,
+// one per item. Record j of the slice is at index slice_rec(j) + s.
+struct SliceRecs {
+  long long x0;   // first item of the slice
+  int cf;         // first producer (T >= C)
+  int n;          // records
+  bool per_item;  // T < C
+};
+__device__ __forceinline__ SliceRecs slice_recs(const long long* pre, int s, long long T, int C) {
+  SliceRecs r{pre[s], 0, 0, T < C};
+  const long long x1 = pre[s + 1];
+  if (x1 <= r.x0) return r;
+  if (r.per_item) {
+    r.n = static_cast<int>(x1 - r.x0);
+  } else {
+    r.cf = cta_of(r.x0, T, C);
+    r.n = cta_of(x1 - 1, T, C) - r.cf + 1;
   }
-  cf = cta_of(pre[s], T, C);
-  cl = cta_of(pre[s + 1] - 1, T, C);
+  return r;
+}
+__device__ __forceinline__ int slice_rec(const SliceRecs& r, long long T, int C, int j) {
+  return r.per_item ? cta_of(r.x0 + j, T, C) : r.cf + j;
 }
 
 // ============================================================ budget
@@ -1428,14 +1120,13 @@ __device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
   constexpr int REC = G * (2 + D);
   __shared__ float s_w[32][G];
   const long long T = P.pre_det[2 * P.units];
-  int cf0, cl0, cf1, cl1;
-  slice_ctas(P.pre_det, 2 * u, T, P.CD, cf0, cl0);
-  slice_ctas(P.pre_det, 2 * u + 1, T, P.CD, cf1, cl1);
-  const int n0 = max(0, cl0 - cf0 + 1), n1 = max(0, cl1 - cf1 + 1);
+  const SliceRecs r0 = slice_recs(P.pre_det, 2 * u, T, P.CD);
+  const SliceRecs r1 = slice_recs(P.pre_det, 2 * u + 1, T, P.CD);
   float m = -INFINITY;
-  for (int x = threadIdx.x; x < (n0 + n1) * G; x += blockDim.x) {
+  for (int x = threadIdx.x; x < (r0.n + r1.n) * G; x += blockDim.x) {
     const int r = x / G, g = x % G;
-    const size_t id = r < n0 ? static_cast<size_t>(cf0 + r + 2 * u) : static_cast<size_t>(cf1 + (r - n0) + 2 * u + 1);
+    const size_t id = r < r0.n ? static_cast<size_t>(slice_rec(r0, T, P.CD, r) + 2 * u)
+                               : static_cast<size_t>(slice_rec(r1, T, P.CD, r - r0.n) + 2 * u + 1);
     m = fmaxf(m, P.rec_det[id * REC + g * (2 + D)]);
   }
 #pragma unroll
@@ -1453,9 +1144,11 @@ __device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
 
 // out = (A_0 + w A_1) / (L_0 + w L_1) for unit u, head g from its records,
 // with part 1 weighted by w = N_tail / b when the tail was sampled (1
-// otherwise). Block of kCombGroups * D threads: thread (r, e) folds every
-// kCombGroups-th record of each list with a running maximum (batches of
-// loads issued ahead of the fold), and the groups' states are then merged.
+// otherwise). Block of groups * D threads (groups = blockDim.x / D, at most
+// kCombGroups): thread (r, e) folds every groups-th record of each slice with
+// a running maximum (batches of loads issued ahead of the fold), and the
+// groups' states are then merged. Only the records written in this call are
+// read (slice_recs).
 constexpr int kCombGroups = 8;
 
 template <int D, int G, int MODE>
@@ -1464,6 +1157,7 @@ __device__ void unit_combine(const DevParams& P, int u, int g) {
   __shared__ float s_st[2][kCombGroups][3][D];
   const UnitInfo inf = P.info[u];
   const int b = u / P.Hkv, h = u % P.Hkv;
+  const int groups = static_cast<int>(blockDim.x) / D;
   const int r = threadIdx.x / D, e = threadIdx.x % D;
   const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
   const bool sampled = MODE == kModeSample && inf.mode == 2 && !inf.exhausted;
@@ -1471,18 +1165,18 @@ __device__ void unit_combine(const DevParams& P, int u, int g) {
   for (int part = 0; part < 2; part++) {
     float m = -INFINITY, l = 0.0f, a = 0.0f;
     auto fold = [&](const long long* pre, const float* rec, int C) {
-      int cf, cl;
-      slice_ctas(pre, 2 * u + part, pre[2 * P.units], C, cf, cl);
+      const long long T = pre[2 * P.units];
+      const SliceRecs sr = slice_recs(pre, 2 * u + part, T, C);
       constexpr int B = 4;  // records loaded together, then folded
-      for (int c0 = cf + r; c0 <= cl; c0 += B * kCombGroups) {
+      for (int j0 = r; j0 < sr.n; j0 += B * groups) {
         float rm[B], rl[B], ra[B];
 #pragma unroll
         for (int j = 0; j < B; j++) {
-          const int c = c0 + j * kCombGroups;
+          const int jj = j0 + j * groups;
           rm[j] = -INFINITY;
           rl[j] = ra[j] = 0.0f;
-          if (c <= cl) {
-            const float* q = rec + static_cast<size_t>(c + 2 * u + part) * REC + g * (2 + D);
+          if (jj < sr.n) {
+            const float* q = rec + static_cast<size_t>(slice_rec(sr, T, C, jj) + 2 * u + part) * REC + g * (2 + D);
             rm[j] = q[0];
             rl[j] = q[1];
             ra[j] = q[2 + e];
@@ -1517,10 +1211,12 @@ __device__ void unit_combine(const DevParams& P, int u, int g) {
   for (int part = 0; part < 2; part++) {
     float m = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < kCombGroups; q++) m = fmaxf(m, s_st[part][q][0][e]);
+    for (int q = 0; q < kCombGroups; q++)
+      if (q < groups) m = fmaxf(m, s_st[part][q][0][e]);
     float l = 0.0f, a = 0.0f;
 #pragma unroll
     for (int q = 0; q < kCombGroups; q++) {
+      if (q >= groups) break;
       const float sc = exp_rel(s_st[part][q][0][e], m);
       l += s_st[part][q][1][e] * sc;
       a += s_st[part][q][2][e] * sc;
@@ -1672,7 +1368,7 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
         __syncwarp();  // the stage is free again
       }
       issued += static_cast<unsigned>(nbw);
-      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHistAll);
+      flush_hist(s_hist, P.hist + static_cast<size_t>(u) * kHist1);
     }
     cur = uend;
   }
@@ -1689,7 +1385,7 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
 }
 
 // ============================================================ k_gather
-template <typename T, int D, int G, int MODE>
+template <typename T, int D, int G, int MODE, bool HOSTKV = false>
 __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(const __grid_constant__ DevParams P) {
   using S = GatherShape<T, D, G>;
   constexpr int E = S::E, NC = S::NC, LOGNC = S::LOGNC, RPW = S::RPW, UNR = S::UNR, R = S::R;
@@ -1822,7 +1518,7 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(con
       // memory form runs (a lane starts one when its row does not directly
       // follow the previous lane's)
       int row = lane < nvalid ? (pid * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps) : 0;
-      if (P.kv_host) {
+      if constexpr (HOSTKV) {
         // caches in mapped host memory: the warp reads the block's rows with
         // plain 16-byte loads over the host link (eight in flight per lane),
         // stores them into the stage and completes its phase with a plain
@@ -2149,7 +1845,7 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
 //   ascending (ties at the threshold to the lowest positions, as the key's
 //   low half orders them). The sorted list, kept in shared memory, then
 //   serves the pilot draws (or the whole tail when it is no larger than the
-//   pilot), as k_draws does after the other selections.
+//   pilot), as k_draws does for the rest of the sample.
 constexpr int kSel1Threads = 1024;
 constexpr int kSel1MaxKeys = 45056;
 constexpr int kSel1Cand = kTopkSmem - kHist2;  // candidate slots; with the histogram, the top-k staging
@@ -2188,7 +1884,7 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
     }
     if (tid < head) s_keys[tid] = ordk[tid];
     if (tid < mlen - head - nbody) s_keys[head + nbody + tid] = ordk[head + nbody + tid];
-    const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHistAll;
+    const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHist1;
     for (int x = tid; x < kHist1; x += kSel1Threads) s_hist[x] = h1[x];
     if (tid == 0) {
       s_digit = 0;
@@ -2326,18 +2022,257 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
   grid_dependents_launch();
 }
 
+// ============================================================ k_topk
+// Top-k selection and pilot draws of one unit in one CTA of kTopkThreads, for
+// any middle length. The keys are read from L2 (the score pass wrote them just
+// before) in one ordered pass: digit 1 (key bits 31..21) of the k-th largest
+// key comes from the score pass's histogram; each warp turns 1024 consecutive
+// keys per round into 32 words of two ballots (key above bin d1; key in bin
+// d1), and a block scan over the packed popcounts appends the positions of
+// both kinds to shared-memory lists in position order, while the keys of bin
+// d1 are counted by digit 2. Every key above bin d1 is in the top k. Digit 3
+// and the threshold key then come from the bin-d1 list alone; its members
+// above the threshold, and the lowest-positioned ones equal to it, are
+// compacted in order, and the two ascending lists are merged into sel (and
+// into shared memory for the draws). When a list would overflow its space
+// (e.g. every score equal), a second ordered pass over all keys selects
+// instead. Then the pilot draws (or the whole tail when it is no larger than
+// the pilot), as k_draws does for the sample.
+constexpr int kTopkThreads = 512;
+constexpr int kTopkAbove = 4096;   // positions above bin d1 kept in shared memory
+constexpr int kTopkCand = 8192;    // positions in bin d1
+constexpr int kTopkTaken = 4096;   // bin-d1 positions taken
+constexpr int kTopkList = 6144;    // the merged list, kept for the draws
+constexpr size_t kTopkKernelSmem = static_cast<size_t>(kHist2 + kTopkAbove + kTopkCand + kTopkTaken + kTopkList) * 4;
+
+// Position of v among n ascending values (the count of those below it).
+__device__ __forceinline__ int lower_bound_s(const int* a, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 2) k_topk(DevParams P) {
+  extern __shared__ __align__(16) unsigned char topk_smem[];
+  unsigned* s_hist = reinterpret_cast<unsigned*>(topk_smem);  // [kHist2]
+  int* s_above = reinterpret_cast<int*>(s_hist + kHist2);     // [kTopkAbove]
+  int* s_cand = s_above + kTopkAbove;                         // [kTopkCand]
+  int* s_took = s_cand + kTopkCand;                           // [kTopkTaken]
+  int* s_list = s_took + kTopkTaken;                          // [kTopkList]
+  __shared__ unsigned s_warp[32];
+  __shared__ int s_digit, s_krem;
+  __shared__ unsigned s_round[2];
+  constexpr int NT = kTopkThreads, NWK = NT / 32;
+  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_dependency_wait();
+  const UnitInfo inf = P.info[u];
+  const int* topk = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;  // global copy
+  if (inf.k > 0) {
+    const int mlen = inf.wst - inf.s1, k = inf.k;
+    const unsigned* keys = P.ordk + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+    int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
+    const bool keep = k <= kTopkList;
+    // digit 1 from the score pass's histogram
+    const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHist1;
+    for (int x = tid; x < kHist1; x += NT) s_hist[x] = __ldcg(h1 + x);
+    if (tid == 0) {
+      s_digit = 0;
+      s_krem = k;
+    }
+    __syncthreads();
+    find_digit_bt<kHist1, NT>(s_hist, k, &s_digit, &s_krem, s_warp);
+    const unsigned d1 = static_cast<unsigned>(s_digit);
+    const int krem1 = s_krem;
+    for (int x = tid; x < kHist2; x += NT) s_hist[x] = 0u;
+    __syncthreads();
+
+    // one ordered pass: positions above bin d1, positions in it, digit-2 counts
+    unsigned na = 0, nc = 0;
+    for (int base = 0; base < mlen; base += 1024 * NWK) {
+      const int wb = base + warp * 1024;
+      unsigned wa = 0, wc = 0;
+#pragma unroll
+      for (int half = 0; half < 2; half++) {
+        unsigned o[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+          const int x = wb + (half * 16 + i) * 32 + lane;
+          o[i] = x < mlen ? __ldcg(keys + x) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+          const int x = wb + (half * 16 + i) * 32 + lane;
+          const unsigned dg = o[i] >> 21;
+          const bool in = x < mlen && dg == d1;
+          const unsigned ba = __ballot_sync(0xffffffffu, x < mlen && dg > d1);
+          const unsigned bc = __ballot_sync(0xffffffffu, in);
+          if (in) atomicAdd(&s_hist[(o[i] >> 10) & 2047u], 1u);
+          if (lane == half * 16 + i) {
+            wa = ba;
+            wc = bc;
+          }
+        }
+      }
+      // a round holds at most 1024 * NWK keys, so both counts fit 16 bits
+      const unsigned packed = (static_cast<unsigned>(__popc(wa)) << 16) | static_cast<unsigned>(__popc(wc));
+      const unsigned incl = block_inclusive_scan(packed, s_warp);
+      const unsigned excl = incl - packed;
+      unsigned pa = na + (excl >> 16), pc = nc + (excl & 0xFFFFu);
+      for (unsigned m = wa; m; m &= m - 1u, pa++)
+        if (pa < static_cast<unsigned>(kTopkAbove)) s_above[pa] = wb + lane * 32 + (__ffs(m) - 1);
+      for (unsigned m = wc; m; m &= m - 1u, pc++)
+        if (pc < static_cast<unsigned>(kTopkCand)) s_cand[pc] = wb + lane * 32 + (__ffs(m) - 1);
+      if (tid == NT - 1) {
+        s_round[0] = incl >> 16;
+        s_round[1] = incl & 0xFFFFu;
+      }
+      __syncthreads();
+      na += s_round[0];
+      nc += s_round[1];
+      __syncthreads();
+    }
+    // digit 2
+    find_digit_bt<kHist2, NT>(s_hist, krem1, &s_digit, &s_krem, s_warp);
+    const unsigned pre = d1 << 11 | static_cast<unsigned>(s_digit);
+    const int krem2 = s_krem;
+    // digit 3 over the bin-d1 list (over every key when it overflowed)
+    for (int x = tid; x < kHist3; x += NT) s_hist[x] = 0u;
+    __syncthreads();
+    const bool cand_ok = nc <= static_cast<unsigned>(kTopkCand);
+    if (cand_ok) {
+      for (int i = tid; i < static_cast<int>(nc); i += NT) {
+        const unsigned o = __ldcg(keys + s_cand[i]);
+        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
+      }
+    } else {
+      for (int x = tid; x < mlen; x += NT) {
+        const unsigned o = __ldcg(keys + x);
+        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
+      }
+    }
+    __syncthreads();
+    find_digit_bt<kHist3, NT>(s_hist, krem2, &s_digit, &s_krem, s_warp);
+    const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
+    const unsigned need_eq = static_cast<unsigned>(s_krem);
+    if (tid == 0) {
+      P.info[u].thr = thr;
+      P.info[u].need_eq = static_cast<int>(need_eq);
+    }
+    const int ntake = k - static_cast<int>(na);  // bin-d1 members taken
+    if (cand_ok && na <= static_cast<unsigned>(kTopkAbove) && ntake >= 0 && ntake <= kTopkTaken) {
+      // the bin-d1 members taken, in position order: every one above thr, and
+      // the first need_eq equal to it
+      unsigned eq_seen = 0, taken = 0;
+      for (int base = 0; base < static_cast<int>(nc); base += NT) {
+        const int i = base + tid;
+        const unsigned o = i < static_cast<int>(nc) ? __ldcg(keys + s_cand[i]) : 0u;
+        const unsigned gt = i < static_cast<int>(nc) && o > thr, eq = i < static_cast<int>(nc) && o == thr;
+        const unsigned packed = (gt << 16) | eq;
+        const unsigned incl = block_inclusive_scan(packed, s_warp);
+        const unsigned excl = incl - packed;
+        const unsigned eq_before = eq_seen + (excl & 0xFFFFu);
+        const unsigned at = taken + (excl >> 16) + min(eq_before, need_eq) - min(eq_seen, need_eq);
+        if ((gt || (eq && eq_before < need_eq)) && at < static_cast<unsigned>(kTopkTaken)) s_took[at] = s_cand[i];
+        if (tid == NT - 1) {
+          s_round[0] = incl >> 16;
+          s_round[1] = incl & 0xFFFFu;
+        }
+        __syncthreads();
+        const unsigned rg = s_round[0], re = s_round[1];
+        taken += rg + min(eq_seen + re, need_eq) - min(eq_seen, need_eq);
+        eq_seen += re;
+        __syncthreads();
+      }
+      // merge the two ascending lists
+      for (int i = tid; i < static_cast<int>(na); i += NT) {
+        const int v = s_above[i];
+        const int idx = i + lower_bound_s(s_took, ntake, v);
+        sel[idx] = inf.s1 + v;
+        if (keep) s_list[idx] = inf.s1 + v;
+      }
+      for (int j = tid; j < ntake; j += NT) {
+        const int v = s_took[j];
+        const int idx = j + lower_bound_s(s_above, static_cast<int>(na), v);
+        sel[idx] = inf.s1 + v;
+        if (keep) s_list[idx] = inf.s1 + v;
+      }
+    } else {
+      // ordered compaction over every key: per round, warp w turns keys
+      // [base + 1024 w, base + 1024 (w + 1)) into 32 words (above thr; equal to
+      // it), and block scans over the packed popcounts give each word's place
+      unsigned gt_seen = 0, eq_seen = 0;
+      for (int base = 0; base < mlen; base += 1024 * NWK) {
+        const int wb = base + warp * 1024;
+        unsigned wgt = 0, weq = 0;
+#pragma unroll 4
+        for (int j = 0; j < 32; j++) {
+          const int x = wb + j * 32 + lane;
+          const unsigned o = x < mlen ? __ldcg(keys + x) : 0u;
+          const unsigned bg = __ballot_sync(0xffffffffu, x < mlen && o > thr);
+          const unsigned be = __ballot_sync(0xffffffffu, x < mlen && o == thr);
+          if (lane == j) {
+            wgt = bg;
+            weq = be;
+          }
+        }
+        const unsigned ng = __popc(wgt), ne = __popc(weq);
+        const unsigned incl = block_inclusive_scan((ng << 16) | ne, s_warp);
+        const unsigned excl = incl - ((ng << 16) | ne);
+        const unsigned gt_before = gt_seen + (excl >> 16), eq_before = eq_seen + (excl & 0xFFFFu);
+        const unsigned keepn = need_eq > eq_before ? min(ne, need_eq - eq_before) : 0u;
+        unsigned wsel = wgt, e = weq;
+        for (unsigned c = 0; c < keepn; c++) {  // the lowest keepn tied positions
+          wsel |= e & (0u - e);
+          e &= e - 1u;
+        }
+        unsigned pos = gt_before + min(eq_before, need_eq);
+        while (wsel) {
+          const int j = inf.s1 + wb + lane * 32 + (__ffs(wsel) - 1);
+          sel[pos] = j;
+          if (keep) s_list[pos] = j;
+          pos++;
+          wsel &= wsel - 1u;
+        }
+        if (tid == NT - 1) {
+          s_round[0] = incl & 0xFFFFu;
+          s_round[1] = incl >> 16;
+        }
+        __syncthreads();
+        eq_seen += s_round[0];
+        gt_seen += s_round[1];
+        __syncthreads();
+      }
+    }
+    __syncthreads();  // the list is complete (shared memory, and the global copy for this CTA)
+    if (keep) topk = s_list;
+  }
+
+  // pilot draws (mode 2), or the whole tail when it is no larger than the pilot (mode 1)
+  const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
+  const bool whole = inf.mode == 1;
+  int* dsel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
+  // the draw counter names the sequence and KV head in the whole batch (a
+  // shard adds its offsets), so a shard draws what the whole batch would
+  const unsigned bb = static_cast<unsigned>(P.batch_offset + u / P.Hkv),
+                 hh = static_cast<unsigned>(P.head_offset + u % P.Hkv);
+  for (int t = tid; t < t1; t += NT) {
+    const int rho = whole ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
+    dsel[t] = tail_position(topk, inf.k, inf.s1, rho);
+  }
+  grid_dependents_launch();
+}
+
 // ============================================================ k_draws
-// Positions of sampled entries. PHASE 0: the pilot draws (or the whole tail
-// when it is no larger than the pilot), after the cluster or grid-wide top-k
-// selection (k_select1 does this itself). PHASE 1, after the budget: draws t
-// in [p, b), or the whole tail when the budget covers it; CTA (0, 0) also
-// writes the sample gather's slice prefix (every budget is known by now).
-// Grid (units, splits).
-template <int PHASE>
+// Positions of the sample's entries after the budget: draws t in [p, b), or
+// the whole tail when the budget covers it; CTA (0, 0) also writes the sample
+// gather's slice prefix (every budget is known by now). Grid (units, splits).
 __global__ void __launch_bounds__(128) k_draws(DevParams P) {
   __shared__ int s_topk[kTopkSmem];
   grid_dependency_wait();
-  if (PHASE == 1 && blockIdx.x == 0 && blockIdx.y == 0) {
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
     __shared__ unsigned s_warp[32];
     __shared__ long long s_carry;
     write_slice_prefix<kModeSample>(P, P.pre_samp, s_warp, &s_carry);
@@ -2347,10 +2282,7 @@ __global__ void __launch_bounds__(128) k_draws(DevParams P) {
   const UnitInfo inf = P.info[u];
   int t0 = 0, t1 = 0;
   bool whole = false;
-  if (PHASE == 0) {
-    t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
-    whole = inf.mode == 1;
-  } else if (inf.mode == 2) {
+  if (inf.mode == 2) {
     whole = inf.exhausted != 0;
     t0 = whole ? 0 : inf.p;
     t1 = whole ? inf.ntail : inf.bsz;
@@ -2540,7 +2472,7 @@ __global__ void __launch_bounds__(kNumThreads) k_numstats(DevParams P) {
 }
 
 // ============================================================ k_combine
-// One CTA per (unit, head), kCombGroups threads per dimension: merge the
+// One CTA per (unit, head), up to kCombGroups threads per dimension: merge the
 // unit's records and write the output.
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kCombGroups * D) k_combine(DevParams P) {
