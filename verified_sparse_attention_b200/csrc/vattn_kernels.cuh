@@ -254,16 +254,23 @@ __global__ void __launch_bounds__(128) k_prep(DevParams P) {
     }
   } else if (P.proxy == kProxyLoki) {
     // projected ranking query: one fused chain over d per component
+    // the head's basis (d x 32 fp32) into shared memory by every thread at
+    // once, then one chain per component over it in order
+    __shared__ float s_basis[D * 32];
+    const float* basis = P.basis + static_cast<size_t>(h) * D * P.rank;
+    const int nb = D * P.rank;  // rank is 32
+    for (int i0 = tid; i0 < nb; i0 += 8 * blockDim.x) {
+      float bv[8];
+#pragma unroll
+      for (int j = 0; j < 8; j++) bv[j] = i0 + j * blockDim.x < nb ? basis[i0 + j * blockDim.x] : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+        if (i0 + j * blockDim.x < nb) s_basis[i0 + j * blockDim.x] = bv[j];
+    }
+    __syncthreads();
     if (tid < P.rank) {
-      // the basis column's loads go out sixteen at a time; the chain stays in order
       float acc = 0.0f;
-      for (int i0 = 0; i0 < D; i0 += 16) {
-        float bv[16];
-#pragma unroll
-        for (int j = 0; j < 16; j++) bv[j] = P.basis[(static_cast<size_t>(h) * D + i0 + j) * P.rank + tid];
-#pragma unroll
-        for (int j = 0; j < 16; j++) acc = __fmaf_rn(s_q[i0 + j], bv[j], acc);
-      }
+      for (int i = 0; i < D; i++) acc = __fmaf_rn(s_q[i], s_basis[i * P.rank + tid], acc);
       P.qsel[static_cast<size_t>(u) * D + tid] = acc;
     }
   }
