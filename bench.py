@@ -461,6 +461,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gqa_32k", choices=list(synth.WORKLOADS))
     ap.add_argument("--eps", type=float, default=None)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per call (default: the workload's own)")
     ap.add_argument("--guarantee", default="denominator", choices=["denominator", "output"],
                     help="what the sample size bounds: the softmax denominator, or the output too")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -482,6 +484,8 @@ def main():
     w = synth.WORKLOADS[args.workload].replace(guarantee=args.guarantee)
     if args.eps is not None:
         w = w.replace(eps=args.eps)
+    if args.batch is not None:
+        w = w.replace(batch=args.batch)
     cfg = {"workload": synth.describe(w), "name": w.name, "batch": w.batch,
            "ctx": w.max_ctx if w.min_ctx == w.max_ctx else [w.min_ctx, w.max_ctx],
            "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
