@@ -427,8 +427,10 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
                                       static_cast<int>(vattn::kSel1Smem)) == cudaSuccess;
   cudaGetLastError();
   if (!ctx->select1 &&
-      cudaFuncSetAttribute(vattn::k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess) {
+      (cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess ||
+       cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreadsFew>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess)) {
     cudaFree(ctx->ws);
     delete ctx;
     return VATTN_ECUDA;
@@ -595,8 +597,12 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   // the middle fits, else streamed from L2 by k_topk
   if (ctx->select1)
     launch(vattn::k_select1, dim3(P.units), dim3(vattn::kSel1Threads), vattn::kSel1Smem, st, P, &launches);
+  else if (P.units <= ctx->num_sms)
+    launch(vattn::k_topk<vattn::kTopkThreadsFew>, dim3(P.units), dim3(vattn::kTopkThreadsFew),
+           vattn::kTopkKernelSmem, st, P, &launches);
   else
-    launch(vattn::k_topk, dim3(P.units), dim3(vattn::kTopkThreads), vattn::kTopkKernelSmem, st, P, &launches);
+    launch(vattn::k_topk<vattn::kTopkThreads>, dim3(P.units), dim3(vattn::kTopkThreads), vattn::kTopkKernelSmem,
+           st, P, &launches);
   launch(P.kv_host ? K.det_host : K.det, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
   if (P.guarantee)
     launch(K.numstats, dim3(P.units, (ctx->G * c.head_dim + vattn::kNumThreads - 1) / vattn::kNumThreads),

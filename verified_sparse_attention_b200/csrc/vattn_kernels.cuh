@@ -2045,7 +2045,8 @@ __global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
 // (e.g. every score equal), a second ordered pass over all keys selects
 // instead. Then the pilot draws (or the whole tail when it is no larger than
 // the pilot), as k_draws does for the sample.
-constexpr int kTopkThreads = 512;
+// threads per CTA: 1024 when every unit has an SM of its own, else 512 (two CTAs per SM)
+constexpr int kTopkThreadsFew = 1024, kTopkThreads = 512;
 constexpr int kTopkAbove = 4096;   // positions above bin d1 kept in shared memory
 constexpr int kTopkCand = 8192;    // positions in bin d1
 constexpr int kTopkTaken = 4096;   // bin-d1 positions taken
@@ -2062,7 +2063,8 @@ __device__ __forceinline__ int lower_bound_s(const int* a, int n, int v) {
   return lo;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 2) k_topk(DevParams P) {
+template <int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) k_topk(DevParams P) {
   extern __shared__ __align__(16) unsigned char topk_smem[];
   unsigned* s_hist = reinterpret_cast<unsigned*>(topk_smem);  // [kHist2]
   int* s_above = reinterpret_cast<int*>(s_hist + kHist2);     // [kTopkAbove]
@@ -2072,7 +2074,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) k_topk(DevParams P) {
   __shared__ unsigned s_warp[32];
   __shared__ int s_digit, s_krem;
   __shared__ unsigned s_round[2];
-  constexpr int NT = kTopkThreads, NWK = NT / 32;
+  constexpr int NWK = NT / 32;
   const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   grid_dependency_wait();
   const UnitInfo inf = P.info[u];
