@@ -27,7 +27,6 @@ struct vattn_ctx {
   int CD = 0, CS = 0;      // record producers (warps) of the det/dense and sample gathers
   size_t gather_smem = 0;   // gathers (all modes)
   int gather_threads = 0;
-  bool select1 = false;     // k_select1 (keys staged in shared memory), else k_topk
   int draw_splits = 1;
   size_t ws_bytes = 0;
   void* ws = nullptr;
@@ -420,17 +419,11 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
     delete ctx;
     return VATTN_ECUDA;
   }
-  // the top-k selection: one CTA per unit with the middle's keys staged in
-  // its shared memory when they fit, else one CTA per unit streaming them
-  ctx->select1 = cfg->max_ctx <= vattn::kSel1MaxKeys &&
-                 cudaFuncSetAttribute(vattn::k_select1, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(vattn::kSel1Smem)) == cudaSuccess;
-  cudaGetLastError();
-  if (!ctx->select1 &&
-      (cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess ||
-       cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreadsFew>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess)) {
+  // the top-k selection (k_topk, two block sizes)
+  if (cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess ||
+      cudaFuncSetAttribute(vattn::k_topk<vattn::kTopkThreadsFew>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(vattn::kTopkKernelSmem)) != cudaSuccess) {
     cudaFree(ctx->ws);
     delete ctx;
     return VATTN_ECUDA;
@@ -593,11 +586,8 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
   }
   // top-p: each unit's top-k size from the mass of its ranking scores
   if (P.topp_den > 0) launch(vattn::k_topp, dim3(P.units), dim3(vattn::kToppThreads), 0, st, P, &launches);
-  // top-k select and pilot draws: keys staged in one CTA's shared memory when
-  // the middle fits, else streamed from L2 by k_topk
-  if (ctx->select1)
-    launch(vattn::k_select1, dim3(P.units), dim3(vattn::kSel1Threads), vattn::kSel1Smem, st, P, &launches);
-  else if (P.units <= ctx->num_sms)
+  // top-k select and pilot draws, one CTA per unit
+  if (P.units <= ctx->num_sms)
     launch(vattn::k_topk<vattn::kTopkThreadsFew>, dim3(P.units), dim3(vattn::kTopkThreadsFew),
            vattn::kTopkKernelSmem, st, P, &launches);
   else

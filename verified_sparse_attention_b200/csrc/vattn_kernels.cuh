@@ -10,8 +10,8 @@
 //                 dim-major K copy); writes the order keys and the histogram
 //                 of their first radix digit
 //   k_topp        (top-p only) each unit's top-k size from its scores' mass
-//   k_select1     top-k select and pilot draws, one CTA per unit, keys staged
-//   k_topk        in shared memory (k_topk: any middle length, keys streamed)
+//   k_topk        top-k select and pilot draws, one CTA per unit, the keys
+//                 streamed from L2
 //   k_gather<det>    gather + softmax-accumulate of I_f and the pilot draws
 //                    (true scores of every query head kept)
 //   k_numstats    (output guarantee only) numerator statistics of the pilot
@@ -1841,197 +1841,9 @@ __device__ void write_draw_positions(const DevParams& P, int u, const UnitInfo& 
   __syncthreads();
 }
 
-// ============================================================ k_select1
-// Top-k selection and pilot draws of one unit in one CTA of 1024 threads,
-// for middles of at most kSel1MaxKeys keys (staged in shared memory by one
-// bulk copy):
-//   digit 1 from the score pass's histogram; one pass over the keys builds
-//   the digit-2 histogram of the keys in bin d1 and collects their indices;
-//   digit 3 is counted over those candidates only (over all keys if they
-//   overflow kSel1Cand); one ordered pass writes the selected positions
-//   ascending (ties at the threshold to the lowest positions, as the key's
-//   low half orders them). The sorted list, kept in shared memory, then
-//   serves the pilot draws (or the whole tail when it is no larger than the
-//   pilot), as k_draws does for the rest of the sample.
-constexpr int kSel1Threads = 1024;
-constexpr int kSel1MaxKeys = 45056;
-constexpr int kSel1Cand = kTopkSmem - kHist2;  // candidate slots; with the histogram, the top-k staging
-constexpr size_t kSel1Smem = static_cast<size_t>(kSel1MaxKeys + 4 + kTopkSmem) * 4;
-
-__global__ void __launch_bounds__(kSel1Threads, 1) k_select1(DevParams P) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned* s_raw = reinterpret_cast<unsigned*>(smem);          // [kSel1MaxKeys + 4]
-  unsigned* s_hist = s_raw + kSel1MaxKeys + 4;                   // [kHist2], then
-  unsigned* s_cand = s_hist + kHist2;                            // [kSel1Cand]; both later the top-k
-  int* s_topk = reinterpret_cast<int*>(s_hist);
-  __shared__ unsigned s_warp[32];
-  __shared__ int s_digit, s_krem;
-  __shared__ unsigned s_ncand;
-  __shared__ __align__(8) uint64_t s_bar;
-  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) mbar_init(&s_bar, 1);
-  mbar_init_fence();
-  __syncthreads();
-  grid_dependency_wait();
-  const UnitInfo inf = P.info[u];
-  const int* topk = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;  // global copy
-  if (inf.k > 0) {
-    const int mlen = inf.wst - inf.s1;
-    const size_t kofs = static_cast<size_t>(u) * P.max_ctx + inf.s1;  // first key in ordk
-    const unsigned* ordk = P.ordk + kofs;
-    // keys at s_keys[0, mlen): s_keys sits at the source's offset within 16
-    // bytes, so the aligned middle of the range is one bulk copy
-    const int shift = static_cast<int>((reinterpret_cast<uintptr_t>(ordk) >> 2) & 3);
-    unsigned* s_keys = s_raw + shift;
-    const int head = min(mlen, (4 - shift) & 3);      // keys before the first 16-byte boundary
-    const int nbody = ((mlen - head) / 4) * 4;         // keys copied in bulk
-    if (tid == 0 && nbody > 0) {
-      mbar_arrive_expect_tx(&s_bar, static_cast<unsigned>(nbody) * 4u);
-      bulk_copy_g2s(s_keys + head, ordk + head, static_cast<unsigned>(nbody) * 4u, &s_bar);
-    }
-    if (tid < head) s_keys[tid] = ordk[tid];
-    if (tid < mlen - head - nbody) s_keys[head + nbody + tid] = ordk[head + nbody + tid];
-    const unsigned* h1 = P.hist + static_cast<size_t>(u) * kHist1;
-    for (int x = tid; x < kHist1; x += kSel1Threads) s_hist[x] = h1[x];
-    if (tid == 0) {
-      s_digit = 0;
-      s_krem = inf.k;
-      s_ncand = 0;
-    }
-    __syncthreads();
-    // digit 1 while the keys are still arriving
-    find_digit_bt<kHist1, kSel1Threads>(s_hist, inf.k, &s_digit, &s_krem, s_warp);
-    const unsigned d1 = static_cast<unsigned>(s_digit);
-    const int krem1 = s_krem;
-    if (nbody > 0 && !__all_sync(0xffffffffu, mbar_wait(&s_bar, 0u)) && lane == 0)
-      atomicOr(P.err, kDevTimeout);
-
-    // digit 2 over the keys of bin d1, collecting them
-    for (int x = tid; x < kHist2; x += kSel1Threads) s_hist[x] = 0u;
-    __syncthreads();  // also: every thread's copy wait is over, the keys are visible
-    for (int x0 = tid; x0 < mlen; x0 += 8 * kSel1Threads) {
-      unsigned o[8];
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int x = x0 + i * kSel1Threads;
-        o[i] = x < mlen ? s_keys[x] : 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int x = x0 + i * kSel1Threads;
-        if (x < mlen && (o[i] >> 21) == d1) {
-          atomicAdd(&s_hist[(o[i] >> 10) & 2047u], 1u);
-          const unsigned slot = atomicAdd(&s_ncand, 1u);
-          if (slot < static_cast<unsigned>(kSel1Cand)) s_cand[slot] = static_cast<unsigned>(x);
-        }
-      }
-    }
-    __syncthreads();
-    find_digit_bt<kHist2, kSel1Threads>(s_hist, krem1, &s_digit, &s_krem, s_warp);
-    const unsigned d2 = static_cast<unsigned>(s_digit);
-    const int krem2 = s_krem;
-    const unsigned ncand = s_ncand;
-
-    // digit 3 over the candidates of prefix (d1, d2)
-    const unsigned pre = d1 << 11 | d2;
-    for (int x = tid; x < kHist3; x += kSel1Threads) s_hist[x] = 0u;
-    __syncthreads();
-    if (ncand <= static_cast<unsigned>(kSel1Cand)) {
-      for (int i = tid; i < static_cast<int>(ncand); i += kSel1Threads) {
-        const unsigned o = s_keys[s_cand[i]];
-        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
-      }
-    } else {
-      for (int x = tid; x < mlen; x += kSel1Threads) {
-        const unsigned o = s_keys[x];
-        if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
-      }
-    }
-    __syncthreads();
-    find_digit_bt<kHist3, kSel1Threads>(s_hist, krem2, &s_digit, &s_krem, s_warp);
-    const unsigned thr = pre << 10 | static_cast<unsigned>(s_digit);
-    const unsigned need_eq = static_cast<unsigned>(s_krem);
-    if (tid == 0) {
-      P.info[u].thr = thr;
-      P.info[u].need_eq = static_cast<int>(need_eq);
-    }
-
-    // ordered compaction through a bitmap: per round, warp w turns keys
-    // [base + 1024 w, base + 1024 (w + 1)) into 32 words (one pair of ballots
-    // per 32 keys; lane j keeps word j). Words follow position order across
-    // threads, so block scans give how many tied keys each word keeps (the
-    // lowest positions) and where its selections go.
-    int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.s1;
-    const bool stage = inf.k <= kTopkSmem;
-    unsigned gt_seen = 0, eq_seen = 0;
-    __shared__ unsigned s_round[2];
-    for (int base = 0; base < mlen; base += 32 * kSel1Threads) {
-      const int wb = base + warp * 1024;
-      unsigned wgt = 0, weq = 0;
-#pragma unroll 8
-      for (int j = 0; j < 32; j++) {
-        const int x = wb + j * 32 + lane;
-        const unsigned o = x < mlen ? s_keys[x] : 0u;
-        const unsigned bg = __ballot_sync(0xffffffffu, x < mlen && o > thr);
-        const unsigned be = __ballot_sync(0xffffffffu, x < mlen && o == thr);
-        if (lane == j) {
-          wgt = bg;
-          weq = be;
-        }
-      }
-      // one scan of (above, tied) counts packed in 16-bit halves (a round
-      // holds at most 32768 keys): a word's selections start at
-      // above_before + min(tied_before, need_eq), and it keeps its lowest
-      // need_eq - tied_before tied positions
-      const unsigned ng = __popc(wgt), ne = __popc(weq);
-      const unsigned incl = block_inclusive_scan((ng << 16) | ne, s_warp);
-      const unsigned excl = incl - ((ng << 16) | ne);
-      const unsigned gt_before = gt_seen + (excl >> 16), eq_before = eq_seen + (excl & 0xFFFFu);
-      const unsigned keep = need_eq > eq_before ? min(ne, need_eq - eq_before) : 0u;
-      unsigned wsel = wgt, e = weq;
-      for (unsigned c = 0; c < keep; c++) {  // the lowest `keep` tied positions
-        wsel |= e & (0u - e);
-        e &= e - 1u;
-      }
-      unsigned pos = gt_before + min(eq_before, need_eq);
-      while (wsel) {
-        const int j = inf.s1 + wb + lane * 32 + (__ffs(wsel) - 1);
-        sel[pos] = j;
-        if (stage) s_topk[pos] = j;
-        pos++;
-        wsel &= wsel - 1u;
-      }
-      if (tid == kSel1Threads - 1) {  // round totals: the last thread holds the inclusive sums
-        s_round[0] = incl & 0xFFFFu;
-        s_round[1] = incl >> 16;
-      }
-      __syncthreads();
-      eq_seen += s_round[0];
-      gt_seen += s_round[1];
-      __syncthreads();
-    }
-    __syncthreads();  // the staged list is complete
-    if (stage) topk = s_topk;
-  }
-
-  // pilot draws (mode 2), or the whole tail when it is no larger than the pilot (mode 1)
-  const int t1 = inf.mode == 2 ? inf.p : (inf.mode == 1 ? inf.ntail : 0);
-  const bool whole = inf.mode == 1;
-  int* dsel = P.sel + static_cast<size_t>(u) * P.max_ctx + inf.nI;
-  // the draw counter names the sequence and KV head in the whole batch (a
-  // shard adds its offsets), so a shard draws what the whole batch would
-  const unsigned bb = static_cast<unsigned>(P.batch_offset + u / P.Hkv),
-                 hh = static_cast<unsigned>(P.head_offset + u % P.Hkv);
-  for (int t = tid; t < t1; t += kSel1Threads) {
-    const int rho = whole ? t : lemire(draw_word(P.seed, bb, hh, static_cast<unsigned>(t)), inf.ntail);
-    dsel[t] = tail_position(topk, inf.k, inf.s1, rho);
-  }
-  grid_dependents_launch();
-}
-
 // ============================================================ k_topk
-// Top-k selection and pilot draws of one unit in one CTA of kTopkThreads, for
-// any middle length. The keys are read from L2 (the score pass wrote them just
+// Top-k selection and pilot draws of one unit in one CTA (kTopkThreadsFew or
+// kTopkThreads threads), for any middle length. The keys are read from L2 (the score pass wrote them just
 // before) in one ordered pass: digit 1 (key bits 31..21) of the k-th largest
 // key comes from the score pass's histogram; each warp turns 1024 consecutive
 // keys per round into 32 words of two ballots (key above bin d1; key in bin
