@@ -291,13 +291,11 @@ void launch(void (*kern)(DevParams), dim3 grid, dim3 block, size_t smem, cudaStr
   (*count)++;
 }
 
-// Threads of a combine CTA (one per unit and head): eight record groups per
-// dimension while the CTAs fit one wave at two per SM, else two (a wave of
-// 256-thread CTAs).
+// Threads of a combine CTA (one per unit and head): sixteen warps while the
+// CTAs fit one wave at two per SM, else eight.
 int comb_threads(const vattn_ctx* ctx, int units) {
   const long long ctas = static_cast<long long>(units) * ctx->G;
-  const int groups = ctas <= 2LL * ctx->num_sms ? vattn::kCombGroups : 2;
-  return groups * ctx->cfg.head_dim;
+  return (ctas <= 2LL * ctx->num_sms ? vattn::kCombWarps : vattn::kCombWarps / 2) * 32;
 }
 
 int finish(vattn_ctx* ctx, int launches) {

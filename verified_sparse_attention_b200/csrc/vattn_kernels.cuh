@@ -1151,86 +1151,124 @@ __device__ void det_record_max(const DevParams& P, int u, float* s_mh) {
 
 // out = (A_0 + w A_1) / (L_0 + w L_1) for unit u, head g from its records,
 // with part 1 weighted by w = N_tail / b when the tail was sampled (1
-// otherwise). Block of groups * D threads (groups = blockDim.x / D, at most
-// kCombGroups): thread (r, e) folds every groups-th record of each slice with
-// a running maximum (batches of loads issued ahead of the fold), and the
-// groups' states are then merged. Only the records written in this call are
-// read (slice_recs).
-constexpr int kCombGroups = 8;
+// otherwise). The unit's records of both parts (and, for the sample combine,
+// of both gathers) form one list; warp x folds entries x, x + warps, ... with
+// a running maximum per part, each lane holding D / 32 accumulator elements,
+// the loads of a batch of entries issued before they are folded. The warps'
+// states are then merged through shared memory. Only the records written in
+// this call are read (slice_recs).
+constexpr int kCombWarps = 16;
 
 template <int D, int G, int MODE>
 __device__ void unit_combine(const DevParams& P, int u, int g) {
   constexpr int REC = G * (2 + D);
-  __shared__ float s_st[2][kCombGroups][3][D];
+  constexpr int PL = D / 32;                      // accumulator elements per lane
+  constexpr int NF = MODE == kModeSample ? 4 : 2; // record lists: (part, gather)
+  static_assert(PL % 2 == 0, "float2 loads of the accumulators");
+  __shared__ float s_acc[2][kCombWarps][D];
+  __shared__ float s_ml[2][kCombWarps][2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
   const UnitInfo inf = P.info[u];
   const int b = u / P.Hkv, h = u % P.Hkv;
-  const int groups = static_cast<int>(blockDim.x) / D;
-  const int r = threadIdx.x / D, e = threadIdx.x % D;
   const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
   const bool sampled = MODE == kModeSample && inf.mode == 2 && !inf.exhausted;
+  // list f: part f / 2 of the sample (f even) or det (f odd) gather when
+  // sampling, else part f of the det / dense gather; the det gather's part-1
+  // records (the pilot) are dropped when the whole tail is taken
+  const long long Td = P.pre_det[2 * P.units];
+  const long long Ts = MODE == kModeSample ? P.pre_samp[2 * P.units] : 0;
+  SliceRecs sr[NF];
+  int start[NF + 1];
+  start[0] = 0;
 #pragma unroll
-  for (int part = 0; part < 2; part++) {
-    float m = -INFINITY, l = 0.0f, a = 0.0f;
-    auto fold = [&](const long long* pre, const float* rec, int C) {
-      const long long T = pre[2 * P.units];
-      const SliceRecs sr = slice_recs(pre, 2 * u + part, T, C);
-      constexpr int B = 4;  // records loaded together, then folded
-      for (int j0 = r; j0 < sr.n; j0 += B * groups) {
-        float rm[B], rl[B], ra[B];
+  for (int f = 0; f < NF; f++) {
+    const bool smp = MODE == kModeSample && f % 2 == 0;
+    const int part = MODE == kModeSample ? f / 2 : f;
+    sr[f] = slice_recs(smp ? P.pre_samp : P.pre_det, 2 * u + part, smp ? Ts : Td, smp ? P.CS : P.CD);
+    if (MODE == kModeSample && f == 3 && whole_tail) sr[f].n = 0;
+    start[f + 1] = start[f] + sr[f].n;
+  }
+  const int N = start[NF];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f, a0[PL], a1[PL];
 #pragma unroll
-        for (int j = 0; j < B; j++) {
-          const int jj = j0 + j * groups;
-          rm[j] = -INFINITY;
-          rl[j] = ra[j] = 0.0f;
-          if (jj < sr.n) {
-            const float* q = rec + static_cast<size_t>(slice_rec(sr, T, C, jj) + 2 * u + part) * REC + g * (2 + D);
-            rm[j] = q[0];
-            rl[j] = q[1];
-            ra[j] = q[2 + e];
-          }
-        }
+  for (int c = 0; c < PL; c++) a0[c] = a1[c] = 0.0f;
+  constexpr int B = PL > 2 ? 3 : 4;  // entries loaded together, then folded
+  for (int j0 = warp; j0 < N; j0 += B * nwarps) {
+    float rm[B], rl[B];
+    float2 ra[B][PL / 2];
+    int rp[B];
 #pragma unroll
-        for (int j = 0; j < B; j++) {  // an empty record has m = -inf, l = 0, acc = 0
-          const float nm = fmaxf(m, rm[j]);
-          const float so = exp_rel(m, nm), sn = exp_rel(rm[j], nm);
-          l = l * so + rl[j] * sn;
-          a = a * so + ra[j] * sn;
-          m = nm;
+    for (int k = 0; k < B; k++) {
+      const int j = j0 + k * nwarps;  // the same for every lane: branches are warp-uniform
+      rm[k] = -INFINITY;
+      rl[k] = 0.0f;
+      rp[k] = -1;
+#pragma unroll
+      for (int c = 0; c < PL / 2; c++) ra[k][c] = make_float2(0.0f, 0.0f);
+      if (j >= N) continue;
+      const float* base = P.rec_det;
+      long long id = 0;
+#pragma unroll
+      for (int f = 0; f < NF; f++) {
+        if (j >= start[f] && j < start[f + 1]) {
+          const bool smp = MODE == kModeSample && f % 2 == 0;
+          const int part = MODE == kModeSample ? f / 2 : f;
+          id = slice_rec(sr[f], smp ? Ts : Td, smp ? P.CS : P.CD, j - start[f]) + 2 * u + part;
+          base = smp ? P.rec_samp : P.rec_det;
+          rp[k] = part;
         }
       }
-    };
-    if (MODE == kModeSample) {
-      fold(P.pre_samp, P.rec_samp, P.CS);
-      // the det gather's records too (the pilot is dropped when the whole
-      // tail is taken)
-      if (!(part == 1 && whole_tail)) fold(P.pre_det, P.rec_det, P.CD);
-    } else {
-      fold(P.pre_det, P.rec_det, P.CD);
+      const float* q = base + static_cast<size_t>(id) * REC + g * (2 + D);
+      rm[k] = q[0];
+      rl[k] = q[1];
+#pragma unroll
+      for (int c = 0; c < PL / 2; c++) ra[k][c] = *reinterpret_cast<const float2*>(q + 2 + lane * PL + 2 * c);
     }
-    s_st[part][r][0][e] = m;
-    s_st[part][r][1][e] = l;
-    s_st[part][r][2][e] = a;
+#pragma unroll
+    for (int k = 0; k < B; k++) {
+      auto fold = [&](float& ms, float& ls, float (&as)[PL]) {
+        const float nm = fmaxf(ms, rm[k]);
+        const float so = exp_rel(ms, nm), sn = exp_rel(rm[k], nm);
+        ls = ls * so + rl[k] * sn;
+#pragma unroll
+        for (int c = 0; c < PL / 2; c++) {
+          as[2 * c] = as[2 * c] * so + ra[k][c].x * sn;
+          as[2 * c + 1] = as[2 * c + 1] * so + ra[k][c].y * sn;
+        }
+        ms = nm;
+      };
+      if (rp[k] == 0) fold(m0, l0, a0);
+      else if (rp[k] == 1) fold(m1, l1, a1);
+    }
+  }
+  const float m[2] = {m0, m1}, l[2] = {l0, l1};
+#pragma unroll
+  for (int part = 0; part < 2; part++) {
+    if (lane == 0) {
+      s_ml[part][warp][0] = m[part];
+      s_ml[part][warp][1] = l[part];
+    }
+#pragma unroll
+    for (int c = 0; c < PL; c++) s_acc[part][warp][lane * PL + c] = part == 0 ? a0[c] : a1[c];
   }
   __syncthreads();
-  if (r != 0) return;
+  const int e = threadIdx.x;
+  if (e >= D) return;
   float M[2], L[2], A[2];
 #pragma unroll
   for (int part = 0; part < 2; part++) {
-    float m = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < kCombGroups; q++)
-      if (q < groups) m = fmaxf(m, s_st[part][q][0][e]);
-    float l = 0.0f, a = 0.0f;
-#pragma unroll
-    for (int q = 0; q < kCombGroups; q++) {
-      if (q >= groups) break;
-      const float sc = exp_rel(s_st[part][q][0][e], m);
-      l += s_st[part][q][1][e] * sc;
-      a += s_st[part][q][2][e] * sc;
+    float mx = -INFINITY;
+    for (int x = 0; x < nwarps; x++) mx = fmaxf(mx, s_ml[part][x][0]);
+    float ls = 0.0f, as = 0.0f;
+    for (int x = 0; x < nwarps; x++) {
+      const float sc = exp_rel(s_ml[part][x][0], mx);
+      ls += s_ml[part][x][1] * sc;
+      as += s_acc[part][x][e] * sc;
     }
-    M[part] = m;
-    L[part] = l;
-    A[part] = a;
+    M[part] = mx;
+    L[part] = ls;
+    A[part] = as;
   }
   float w = 1.0f;
   if (sampled) w = static_cast<float>(static_cast<double>(inf.ntail) / static_cast<double>(inf.bsz));
@@ -2293,10 +2331,10 @@ __global__ void __launch_bounds__(kNumThreads) k_numstats(DevParams P) {
 }
 
 // ============================================================ k_combine
-// One CTA per (unit, head), up to kCombGroups threads per dimension: merge the
-// unit's records and write the output.
+// One CTA per (unit, head) of D / 32 to kCombWarps warps: merge the unit's
+// records and write the output.
 template <int D, int G, int MODE>
-__global__ void __launch_bounds__(kCombGroups * D) k_combine(DevParams P) {
+__global__ void __launch_bounds__(kCombWarps * 32, 2) k_combine(DevParams P) {
   grid_dependency_wait();
   unit_combine<D, G, MODE>(P, blockIdx.x, blockIdx.y);
   grid_dependents_launch();
