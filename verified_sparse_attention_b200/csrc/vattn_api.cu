@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <vector>
 
 #include "vattn.h"
@@ -116,6 +117,15 @@ int encode_row_maps(const vattn_config& c, const void* k, const void* v, int num
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return VATTN_ECUDA;
   }
+  if (c.dtype == VATTN_BF16) {  // the tensor-core gathers' swizzled half-row boxes
+    const cuuint32_t hbox[2] = {64u, 1u};
+    for (int i = 0; i < 2; i++) {
+      const CUresult r = fn(i ? &P->tmv_sw : &P->tmk_sw, dt, 2, const_cast<void*>(i ? v : k), dims, strides, hbox,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return VATTN_ECUDA;
+    }
+  }
   return VATTN_OK;
 }
 
@@ -134,6 +144,9 @@ struct Kernels {
   void (*det_host)(DevParams);     // the gathers for caches in host memory
   void (*sample_host)(DevParams);
   void (*dense_host)(DevParams);
+  void (*sample_tc)(DevParams);    // tensor-core sample and dense gathers (bf16, device caches)
+  void (*dense_tc)(DevParams);
+  size_t tc_smem;
   void (*budget)(DevParams);
   void (*numstats)(DevParams);
   void (*combine_sample)(DevParams);
@@ -159,6 +172,14 @@ Kernels kernels_for() {
   k.det_host = vattn::k_gather<T, D, G, vattn::kModeDet, true>;
   k.sample_host = vattn::k_gather<T, D, G, vattn::kModeSample, true>;
   k.dense_host = vattn::k_gather<T, D, G, vattn::kModeDense, true>;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    k.sample_tc = vattn::k_gather_tc<D, G, vattn::kModeSample>;
+    k.dense_tc = vattn::k_gather_tc<D, G, vattn::kModeDense>;
+    k.tc_smem = vattn::TcShape<D, G>::SMEM;
+  } else {
+    k.sample_tc = k.dense_tc = nullptr;
+    k.tc_smem = 0;
+  }
   k.budget = vattn::k_budget<D, G>;
   k.numstats = vattn::k_numstats<T, D, G>;
   k.combine_sample = vattn::k_combine<D, G, vattn::kModeSample>;
@@ -364,6 +385,8 @@ int vattn_create(vattn_ctx** out, const vattn_config* cfg) {
   ctx->gather_threads = K.gather_threads;
   for (auto fn : {K.det, K.sample, K.dense, K.det_host, K.sample_host, K.dense_host})
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->gather_smem));
+  for (auto fn : {K.sample_tc, K.dense_tc})
+    if (fn) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(K.tc_smem));
   cudaFuncSetAttribute(K.numstats, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(vattn::kNumSmem));
   int gocc = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&gocc, K.sample, K.gather_threads, ctx->gather_smem);
@@ -597,7 +620,11 @@ int vattn_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const void*
            dim3(vattn::kNumThreads), vattn::kNumSmem, st, P, &launches);
   launch(K.budget, dim3(P.units), dim3(vattn::kBudgetThreads), 0, st, P, &launches);
   launch(vattn::k_draws, dim3(P.units, ctx->draw_splits * 4), dim3(128), 0, st, P, &launches);
-  launch(P.kv_host ? K.sample_host : K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  if (!P.kv_host && K.sample_tc)
+    launch(K.sample_tc, dim3(ctx->gather_grid), dim3(ctx->gather_threads), K.tc_smem, st, P, &launches);
+  else
+    launch(P.kv_host ? K.sample_host : K.sample, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem,
+           st, P, &launches);
   launch(K.combine_sample, dim3(P.units, ctx->G), dim3(comb_threads(ctx, P.units)), 0, st, P, &launches);
   return finish(ctx, launches);
 }
@@ -643,7 +670,11 @@ int vattn_dense_decode(vattn_ctx* ctx, const void* q, const void* k_cache, const
   P.sel = reinterpret_cast<int*>(ctx->ordk);
   int launches = 0;
   launch(K.prep, dim3(P.units + 1), dim3(128), 0, st, P, &launches);
-  launch(P.kv_host ? K.dense_host : K.dense, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem, st, P, &launches);
+  if (!P.kv_host && K.dense_tc)
+    launch(K.dense_tc, dim3(ctx->gather_grid), dim3(ctx->gather_threads), K.tc_smem, st, P, &launches);
+  else
+    launch(P.kv_host ? K.dense_host : K.dense, dim3(ctx->gather_grid), dim3(ctx->gather_threads), ctx->gather_smem,
+           st, P, &launches);
   launch(K.combine_dense, dim3(P.units, ctx->G), dim3(comb_threads(ctx, P.units)), 0, st, P, &launches);
   return finish(ctx, launches);
 }

@@ -47,6 +47,9 @@ struct DevParams {
   // 2-D row maps of the K and V caches ([rows][D], one-row boxes) for the
   // row-gathering tensor copies; rows = num_pages * Hkv * page_size
   CUtensorMap tmk, tmv;
+  // the same views in boxes of one row by 64 columns with the 128-byte
+  // swizzle, for the tensor-core gathers (bf16 caches in device memory)
+  CUtensorMap tmk_sw, tmv_sw;
   // shapes
   int Hq, Hkv, G, D;
   int pps;        // page-table entries per sequence

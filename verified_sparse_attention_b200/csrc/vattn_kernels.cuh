@@ -655,8 +655,15 @@ struct TReduce {
 };
 
 // CTA of C holding flattened item x of T (CTA c owns [c*T/C, (c+1)*T/C)).
+// floor(num / den) for num >= 0, den > 0: a 32-bit division when both fit
+// (the common case), else the 64-bit one
+__device__ __forceinline__ long long div_nonneg(long long num, long long den) {
+  if (static_cast<unsigned long long>(num | den) <= 0xFFFFFFFFull)
+    return static_cast<long long>(static_cast<unsigned>(num) / static_cast<unsigned>(den));
+  return num / den;
+}
 __device__ __forceinline__ int cta_of(long long x, long long T, int C) {
-  return static_cast<int>(((x + 1) * C - 1) / T);
+  return static_cast<int>(div_nonneg((x + 1) * C - 1, T));
 }
 
 // Item counts of unit u's two slices in a mode (from its validated state).
@@ -1458,14 +1465,14 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(con
   float* rec = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
   const int W = gridDim.x * NW, gw = blockIdx.x * NW + warp;
   const long long Tt = pre[2 * P.units];
-  const long long cbeg = Tt * (blockIdx.x * NW) / W, cend = Tt * ((blockIdx.x + 1) * NW) / W;
+  const long long cbeg = div_nonneg(Tt * (blockIdx.x * NW), W), cend = div_nonneg(Tt * ((blockIdx.x + 1) * NW), W);
   // the CTA's first slice: the one non-empty slice holding item cbeg
   if (cbeg < cend)
     for (int s = threadIdx.x; s < 2 * P.units; s += blockDim.x)
       if (pre[s] <= cbeg && cbeg < pre[s + 1]) s_first = s;
   __syncthreads();
   int sidx = s_first;
-  const long long wbeg = Tt * gw / W, wend = Tt * (gw + 1) / W;
+  const long long wbeg = div_nonneg(Tt * gw, W), wend = div_nonneg(Tt * (gw + 1), W);
   long long cur = wbeg;
   const T* kc = static_cast<const T*>(P.k);
   const T* vc = static_cast<const T*>(P.v);
@@ -1823,6 +1830,328 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(con
     __syncwarp();  // s_ll is reused by the next slice
     cur = send;
   }
+  grid_dependents_launch();
+}
+
+// ============================================================ k_gather_tc
+// The sample and dense gathers for bf16 caches in device memory, on the
+// tensor cores. The streaming scheme is k_gather's (persistent grid, every
+// warp a record producer over a contiguous item range, a private ring of
+// stages filled NS - 1 blocks ahead, bounded mbarrier waits), but every row
+// arrives through tile::gather4 copies of 128-byte half rows with the 128-byte
+// swizzle (the 16-byte chunk index within a half row XORed with the row's
+// index mod 8), so the fragment loads of eight rows touch eight different
+// bank groups. Per block of 16 rows: the scores S[r][g] = K[r] . q_g as
+// D / 16 bf16 MMAs (m16n8k16, the group's heads in the 8 columns, fp32
+// accumulation), the online softmax in the accumulator layout (each lane holds
+// heads 2 (lane % 4) and 2 (lane % 4) + 1 of rows lane / 4 and lane / 4 + 8),
+// then O^T[d][g] += V^T[d][r] P[r][g] as D / 16 MMAs per term of the weights
+// split into two bf16 terms (hi = bf16(p), lo = bf16(p - hi): 2^-16 relative),
+// the weights' fragment transposed into the operand layout by movmatrix. The
+// output accumulator has the same columns as the scores, so rescaling by a new
+// running maximum needs no exchange between lanes. The records are
+// k_gather's: (m, l, acc[D]) per head.
+template <int D, int G>
+struct TcShape {
+  static constexpr int R = 16;                     // rows per block
+  static constexpr int H = D / 64;                 // 128-byte halves of a row
+  static constexpr int HALF = R * 128;             // bytes of one half of a block's rows
+  static constexpr int MATB = H * HALF;            // the block's K (or V) rows
+  static constexpr int BLKB = 2 * MATB;            // K, then V
+  static constexpr int NW = 8;                     // warps per CTA
+  static constexpr int NS = (192 * 1024) / (NW * BLKB);  // stages filling a 192 KB ring
+  static constexpr int KT = D / 16;                // k-steps of a score tile; M-tiles of the output
+  static constexpr int REC = G * (2 + D);
+  static constexpr size_t RING = static_cast<size_t>(NW) * NS * BLKB;
+  static constexpr size_t OFF_BAR = RING;
+  static constexpr size_t SMEM = 1024 + OFF_BAR + static_cast<size_t>(NW) * NS * 8;  // 1 KB to align the ring
+  static_assert(G <= 8, "the group's heads fit the 8 columns of a score tile");
+  static_assert(D % 64 == 0, "whole 128-byte half rows");
+  static_assert(SMEM <= 227 * 1024, "tensor-core gather shared memory");
+};
+
+// Byte offset of 16-byte chunk ch of row r in a swizzled [16 rows][D] bf16
+// tile (halves of 16 x 128 bytes, 1024-byte aligned).
+__device__ __forceinline__ unsigned tc_off(int r, int ch) {
+  return static_cast<unsigned>((ch >> 3) * (16 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void ldsm_x4(unsigned addr, unsigned (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(unsigned addr, unsigned (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ unsigned movm_t(unsigned x) {
+  unsigned y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const unsigned (&a)[4], unsigned b0, unsigned b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// two floats as bf16 (first in the low half), rounded to nearest
+__device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const unsigned*>(&v);
+}
+// (hi, lo) bf16 terms of two weights: p = hi + lo to 2^-16 relative
+__device__ __forceinline__ void split_bf16x2(float p0, float p1, unsigned& hi, unsigned& lo) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
+  hi = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+  lo = pack_bf16x2(p0 - __bfloat162float(h0), p1 - __bfloat162float(h1));
+}
+// tile::gather4 copy of four rows' columns [x, x + box) into shared memory
+__device__ __forceinline__ void gather4x_g2s(void* dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
+                                             int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
+template <int D, int G, int MODE>
+__global__ void __launch_bounds__(TcShape<D, G>::NW * 32, 1) k_gather_tc(const __grid_constant__ DevParams P) {
+  using S = TcShape<D, G>;
+  constexpr int R = S::R, H = S::H, HALF = S::HALF, MATB = S::MATB, BLKB = S::BLKB, NW = S::NW, NS = S::NS,
+                KT = S::KT, REC = S::REC;
+  static_assert(MODE == kModeSample || MODE == kModeDense, "sample and dense gathers");
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR) + warp * NS;
+  unsigned char* ring = smem + static_cast<size_t>(warp) * NS * BLKB;
+  const unsigned ring_s = smem_u32(ring);
+
+  __shared__ int s_first;
+  if (lane < NS) mbar_init(&bars[lane], 1);
+  if (threadIdx.x == 0) s_first = 0;
+  mbar_init_fence();
+  __syncthreads();
+  grid_dependency_wait();
+
+  // every warp is a record producer: warp gw of W owns items [T*gw/W, T*(gw+1)/W)
+  const long long* pre = (MODE == kModeSample) ? P.pre_samp : P.pre_det;
+  float* rec = (MODE == kModeSample) ? P.rec_samp : P.rec_det;
+  const int W = gridDim.x * NW, gw = blockIdx.x * NW + warp;
+  const long long Tt = pre[2 * P.units];
+  const long long cbeg = div_nonneg(Tt * (blockIdx.x * NW), W), cend = div_nonneg(Tt * ((blockIdx.x + 1) * NW), W);
+  if (cbeg < cend)
+    for (int s = threadIdx.x; s < 2 * P.units; s += blockDim.x)
+      if (pre[s] <= cbeg && cbeg < pre[s + 1]) s_first = s;
+  __syncthreads();
+  int sidx = s_first;
+  const long long wbeg = div_nonneg(Tt * gw, W), wend = div_nonneg(Tt * (gw + 1), W);
+  long long cur = wbeg;
+  unsigned issued = 0;  // blocks this warp issued in earlier slices (stage and phase follow from it)
+  bool failed = false;
+  // fragment addresses: lane i serves matrix i / 8, row i % 8 of an ldmatrix.x4
+  const int fj = lane >> 3, fr = lane & 7;
+  const int hc = 2 * (lane & 3);  // this lane's two head columns
+
+  while (cur < wend) {
+    while (pre[sidx + 1] <= cur) sidx++;
+    const long long send = min(wend, pre[sidx + 1]);
+    const int u = sidx >> 1;
+    const int lb = static_cast<int>(cur - pre[sidx]), le = static_cast<int>(send - pre[sidx]);
+    const int b = u / P.Hkv, h = u % P.Hkv;
+    // the query operand: B[k = d][n = head] = q_head[d]; lane holds head lane / 4,
+    // dims 16 kt + 2 (lane % 4) + {0, 1} and those + 8 (zero columns past G)
+    unsigned qf[KT][2];
+    {
+      const int qh = lane >> 2;
+      const unsigned short* qp = static_cast<const unsigned short*>(P.q) +
+                                 (static_cast<size_t>(b) * P.Hq + h * G + (qh < G ? qh : 0)) * D + hc;
+#pragma unroll
+      for (int kt = 0; kt < KT; kt++)
+#pragma unroll
+        for (int x = 0; x < 2; x++) {
+          const unsigned lo = qp[16 * kt + 8 * x], hi = qp[16 * kt + 8 * x + 1];
+          qf[kt][x] = qh < G ? (lo | (hi << 16)) : 0u;
+        }
+    }
+    const UnitInfo inf = P.info[u];
+    const int pid_c = P.pps == 1 ? P.page_table[static_cast<size_t>(b) * P.pps] : 0;
+    const bool valid = inf.n > 0;
+    const int* sel = P.sel + static_cast<size_t>(u) * P.max_ctx;
+    const bool whole_tail = MODE == kModeSample && inf.mode == 2 && inf.exhausted;
+
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    float o[KT][4];
+#pragma unroll
+    for (int mt = 0; mt < KT; mt++)
+#pragma unroll
+      for (int x = 0; x < 4; x++) o[mt][x] = 0.0f;
+
+    const int nitems = valid ? le - lb : 0;
+    const int nblk = (nitems + R - 1) / R;
+    const int nbw = failed ? 0 : nblk;
+    int nis = 0;  // blocks issued in this slice
+
+    // producer side: lane r < R owns row r of a block
+    auto pos_of = [&](int t) -> int {
+      const int x = t * R + lane;
+      if (t >= nbw || lane >= R || x >= nitems) return -1;
+      if (MODE == kModeDense) return lb + x;
+      return sel[inf.nI + (whole_tail ? lb + x : inf.p + lb + x)];
+    };
+    auto pid_of = [&](int pos) -> int {
+      if (P.pps == 1) return pid_c;
+      return pos < 0 ? 0 : P.page_table[static_cast<size_t>(b) * P.pps + page_slot(P, pos)];
+    };
+    auto issue = [&](int t, int pos, int pid) {
+      const unsigned g = issued + static_cast<unsigned>(t);
+      const int st = static_cast<int>(g % NS);
+      const int nvalid = min(R, nitems - t * R);
+      unsigned char* dst = ring + st * BLKB;
+      fence_proxy_async();
+      nis++;
+      // rows past the end repeat row 0 (finite values under zero weights)
+      int row = lane < nvalid ? (pid * P.Hkv + h) * P.ps + (pos - page_slot(P, pos) * P.ps) : 0;
+      const int row0v = __shfl_sync(0xffffffffu, row, 0);
+      if (lane >= nvalid) row = row0v;
+      const int r1 = __shfl_down_sync(0xffffffffu, row, 1);
+      const int r2 = __shfl_down_sync(0xffffffffu, row, 2);
+      const int r3 = __shfl_down_sync(0xffffffffu, row, 3);
+      if (lane == 0) mbar_arrive_expect_tx(&bars[st], static_cast<unsigned>(BLKB));
+      __syncwarp();
+      if (lane < R && (lane & 3) == 0) {
+#pragma unroll
+        for (int hf = 0; hf < H; hf++) {
+          gather4x_g2s(dst + hf * HALF + lane * 128, &P.tmk_sw, hf * 64, row, r1, r2, r3, &bars[st]);
+          gather4x_g2s(dst + MATB + hf * HALF + lane * 128, &P.tmv_sw, hf * 64, row, r1, r2, r3, &bars[st]);
+        }
+      }
+    };
+
+    // fill the ring; the address pipeline then runs one and two blocks ahead
+    // of the issue (page ids for block t + NS - 1, positions for t + NS)
+    int posA;
+    {
+      int posq[NS], pidq[NS - 1];
+#pragma unroll
+      for (int t = 0; t < NS; t++) posq[t] = pos_of(t);
+#pragma unroll
+      for (int t = 0; t < NS - 1; t++) pidq[t] = pid_of(posq[t]);
+#pragma unroll
+      for (int t = 0; t < NS - 1; t++)
+        if (t < nbw) issue(t, posq[t], pidq[t]);
+      posA = posq[NS - 1];
+    }
+    int pidA = pid_of(posA);
+    int posB = pos_of(NS);
+
+#pragma unroll 1
+    for (int t = 0; t < nbw; t++) {
+      if (t + NS - 1 < nbw && !failed) issue(t + NS - 1, posA, pidA);
+      posA = posB;
+      pidA = pid_of(posA);
+      posB = pos_of(t + NS + 1);
+
+      if (t >= nis) continue;  // never issued (only after a failed wait)
+      const unsigned g = issued + static_cast<unsigned>(t);
+      const int st = static_cast<int>(g % NS);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
+        if (!failed && lane == 0) atomicOr(P.err, static_cast<unsigned>(kDevTimeout));
+        failed = true;
+      }
+      if (failed) continue;
+      const unsigned kb = ring_s + static_cast<unsigned>(st * BLKB), vb = kb + MATB;
+
+      // scores: S[r][head] over D / 16 k-steps
+      float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int kt = 0; kt < KT; kt++) {
+        unsigned a[4];
+        ldsm_x4(kb + tc_off(((fj & 1) << 3) | fr, 2 * kt + (fj >> 1)), a);
+        mma_bf16(sc, a, qf[kt][0], qf[kt][1]);
+      }
+      // online softmax: rows lane / 4 (values 0, 1) and lane / 4 + 8 (2, 3)
+      const int nvalid = min(R, nitems - t * R);
+      const int ra = lane >> 2;
+      float sv[4];
+#pragma unroll
+      for (int x = 0; x < 4; x++) sv[x] = (ra + (x >> 1) * 8) < nvalid ? sc[x] * P.scale : -INFINITY;
+      float bm[2] = {fmaxf(sv[0], sv[2]), fmaxf(sv[1], sv[3])};
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int k = 0; k < 2; k++) bm[k] = fmaxf(bm[k], __shfl_xor_sync(0xffffffffu, bm[k], off));
+      float cf[2];
+#pragma unroll
+      for (int k = 0; k < 2; k++) {
+        const float nm = fmaxf(m_run[k], bm[k]);
+        cf[k] = exp_rel(m_run[k], nm);
+        m_run[k] = nm;
+      }
+      float pv[4];
+#pragma unroll
+      for (int x = 0; x < 4; x++) pv[x] = sv[x] == -INFINITY ? 0.0f : __expf(sv[x] - m_run[x & 1]);
+#pragma unroll
+      for (int k = 0; k < 2; k++) l_run[k] = l_run[k] * cf[k] + (pv[k] + pv[2 + k]);
+      if (__any_sync(0xffffffffu, cf[0] != 1.0f || cf[1] != 1.0f)) {
+#pragma unroll
+        for (int mt = 0; mt < KT; mt++)
+#pragma unroll
+          for (int x = 0; x < 4; x++) o[mt][x] *= cf[x & 1];
+      }
+      // the weights as the B operand B[k = r][n = head]: transposes of the
+      // [r][head-pair] fragments of rows 0-7 and 8-15
+      unsigned ph0, pl0, ph1, pl1;
+      split_bf16x2(pv[0], pv[1], ph0, pl0);
+      split_bf16x2(pv[2], pv[3], ph1, pl1);
+      ph0 = movm_t(ph0);
+      pl0 = movm_t(pl0);
+      ph1 = movm_t(ph1);
+      pl1 = movm_t(pl1);
+      // O^T[d][head] += V^T[d][r] P[r][head], one M-tile of 16 dims at a time
+#pragma unroll
+      for (int mt = 0; mt < KT; mt++) {
+        unsigned a[4];
+        ldsm_x4_t(vb + tc_off(((fj >> 1) << 3) | fr, 2 * mt + (fj & 1)), a);
+        mma_bf16(o[mt], a, ph0, ph1);
+        mma_bf16(o[mt], a, pl0, pl1);
+      }
+      __syncwarp();  // the stage is free again
+    }
+    issued += static_cast<unsigned>(nbw);
+
+    // ---- this warp's record for the slice: (m, l, acc[D]) per head; lane
+    // holds dims 16 mt + lane / 4 (+ 8) of heads hc, hc + 1
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+      for (int k = 0; k < 2; k++) l_run[k] += __shfl_xor_sync(0xffffffffu, l_run[k], off);
+    float* r = rec + static_cast<size_t>(gw + sidx) * REC;
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+      const int hh = hc + k;
+      if (hh >= G) continue;
+      float* rh = r + hh * (2 + D);
+      if (lane < 4) {
+        rh[0] = m_run[k];
+        rh[1] = l_run[k];
+      }
+#pragma unroll
+      for (int mt = 0; mt < KT; mt++) {
+        rh[2 + 16 * mt + (lane >> 2)] = o[mt][k];
+        rh[2 + 16 * mt + (lane >> 2) + 8] = o[mt][2 + k];
+      }
+    }
+    __syncwarp();
+    cur = send;
+  }
+
   grid_dependents_launch();
 }
 
