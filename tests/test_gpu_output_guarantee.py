@@ -81,7 +81,7 @@ def test_edge_lengths_paged():
     check(w, inputs=cpu)
 
 
-def test_full_size_gqa_32k_sampled_units():
+def test_full_size_gqa_32k_every_unit():
     _full_check(_out(W["gqa_32k"], eps=0.5))
 
 

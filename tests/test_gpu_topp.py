@@ -96,7 +96,7 @@ def test_long_context_streamed_select():
     check(_p(synth.scaled(W["gqa_32k"], max_ctx=50000, batch=1, num_q_heads=8, num_kv_heads=2), 4, 5))
 
 
-def test_full_size_gqa_32k_sampled_units():
+def test_full_size_gqa_32k_every_unit():
     _full_check(_p(W["gqa_32k"], 9, 10))
 
 

@@ -581,10 +581,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned by
 // Bounded wait for the completion of the barrier phase with parity `parity`;
 // false when `tries` tries ran out (each try may itself suspend for a while,
 // so the default limit ends a wait that can never complete in about a second).
-// A kernel whose wait failed issues no further copies into the ring; copies it
-// had issued before may still be landing in its shared memory when it exits,
-// the one hazard left after a timeout (it can only follow a copy that never
-// completes, which the row bounds of every copy rule out in normal operation).
+// A warp whose wait failed issues no further copies into its ring and first
+// waits once more, with the same limit, for every block it still has in
+// flight (drain_ring), so that no copy lands in shared memory after it has
+// moved on; a wait can only fail after a copy that never completes, which the
+// row bounds of every copy rule out in normal operation.
 constexpr int kWaitTries = 1 << 20;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, int tries = kWaitTries) {
   const unsigned a = smem_u32(bar);
@@ -601,6 +602,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, int tr
 }
 // Orders this thread's earlier generic shared-memory accesses before later
 // async-proxy writes (a bulk copy into a stage that was just read).
+// Bounded waits for blocks [t, nis) of a slice (ring stage and phase from
+// the running block count issued + t), after the wait on block t failed.
+__device__ __noinline__ void drain_ring(uint64_t* bars, int NS, unsigned issued, int t, int nis) {
+  for (int t2 = t; t2 < nis; t2++) {
+    const unsigned g = issued + static_cast<unsigned>(t2);
+    mbar_wait(&bars[g % NS], (g / NS) & 1u);
+  }
+}
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -1394,6 +1403,7 @@ __global__ void __launch_bounds__(ScoreShape<T, W>::NW * 32, 1) k_score_tma(DevP
         if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
           if (!failed && lane == 0) atomicOr(P.err, kDevTimeout);
           failed = true;
+          drain_ring(bars, NS, issued, t, nis);
         }
         if (failed) continue;
         const unsigned char* sb = ring + st * S::BLKB;
@@ -1671,6 +1681,7 @@ __global__ void __launch_bounds__(GatherShape<T, D, G>::NW * 32, 1) k_gather(con
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
         if (!failed && lane == 0) atomicOr(P.err, static_cast<unsigned>(kDevTimeout));
         failed = true;
+        drain_ring(bars, NS, issued, t, nis);
       }
       if (failed) continue;
       const unsigned char* kb = ring + st * S::BLKB;
@@ -2064,6 +2075,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NW * 32, 1) k_gather_tc(const _
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], (g / NS) & 1u))) {
         if (!failed && lane == 0) atomicOr(P.err, static_cast<unsigned>(kDevTimeout));
         failed = true;
+        drain_ring(bars, NS, issued, t, nis);
       }
       if (failed) continue;
       const unsigned kb = ring_s + static_cast<unsigned>(st * BLKB), vb = kb + MATB;
