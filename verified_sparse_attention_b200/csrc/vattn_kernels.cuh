@@ -788,9 +788,21 @@ __device__ __forceinline__ U128 warp_sum_u128(U128 v) {
 // (p (p - 1)) and D = S_f + N_tail * S1 / p, in double in a fixed operation
 // order. b = max(p, max_h n_h); b >= N_tail takes the whole tail instead.
 // Block of up to 1024 threads.
+constexpr int kBudgetBatch = 4;  // items per thread whose scores are loaded together
+// The first batch of thread t's scores (items t + k * threads, k < kBudgetBatch),
+// loaded by the caller before the score maxima are known.
+template <int G>
+__device__ __forceinline__ void load_budget_batch(const float* ps, int nA, float (&sv)[kBudgetBatch][G]) {
+#pragma unroll
+  for (int k = 0; k < kBudgetBatch; k++) {
+    const int i = static_cast<int>(threadIdx.x) + k * static_cast<int>(blockDim.x);
+#pragma unroll
+    for (int g = 0; g < G; g++) sv[k][g] = i < nA ? ps[static_cast<size_t>(i) * G + g] : 0.0f;
+  }
+}
 template <int G>
 __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, const float* ps,
-                            const float* s_mh) {
+                            const float* s_mh, const float (&first)[kBudgetBatch][G]) {
   __shared__ unsigned long long s_a[32][G], s_b[32][G];
   __shared__ U128 s_c[32][G];
   __shared__ int s_need[G];
@@ -821,15 +833,22 @@ __device__ void unit_budget(const DevParams& P, int u, const UnitInfo& inf, cons
     sf[g] = s1[g] = 0ull;
     s2[g] = U128{0ull, 0ull};
   }
-  constexpr int BATCH = 4;
+  constexpr int BATCH = kBudgetBatch;
   const int nt = blockDim.x;
   for (int i0 = tid; i0 < nA; i0 += BATCH * nt) {
     float sv[BATCH][G];
+    if (i0 == tid) {  // the first batch arrived with the call
 #pragma unroll
-    for (int k = 0; k < BATCH; k++) {
-      const int i = i0 + k * nt;
+      for (int k = 0; k < BATCH; k++)
 #pragma unroll
-      for (int g = 0; g < G; g++) sv[k][g] = i < nA ? ps[static_cast<size_t>(i) * G + g] : 0.0f;
+        for (int g = 0; g < G; g++) sv[k][g] = first[k][g];
+    } else {
+#pragma unroll
+      for (int k = 0; k < BATCH; k++) {
+        const int i = i0 + k * nt;
+#pragma unroll
+        for (int g = 0; g < G; g++) sv[k][g] = i < nA ? ps[static_cast<size_t>(i) * G + g] : 0.0f;
+      }
     }
 #pragma unroll
     for (int k = 0; k < BATCH; k++) {
@@ -2345,9 +2364,14 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_topk(DevParams P) {
     for (int x = tid; x < kHist3; x += NT) s_hist[x] = 0u;
     __syncthreads();
     const bool cand_ok = nc <= static_cast<unsigned>(kTopkCand);
+    // the candidates' keys, kept for the compaction in s_list (unused until
+    // the merge) when they fit
+    unsigned* s_ckey = reinterpret_cast<unsigned*>(s_list);
+    const bool ckey = nc <= static_cast<unsigned>(kTopkList);
     if (cand_ok) {
       for (int i = tid; i < static_cast<int>(nc); i += NT) {
         const unsigned o = __ldcg(keys + s_cand[i]);
+        if (ckey) s_ckey[i] = o;
         if ((o >> 10) == pre) atomicAdd(&s_hist[o & 1023u], 1u);
       }
     } else {
@@ -2371,7 +2395,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_topk(DevParams P) {
       unsigned eq_seen = 0, taken = 0;
       for (int base = 0; base < static_cast<int>(nc); base += NT) {
         const int i = base + tid;
-        const unsigned o = i < static_cast<int>(nc) ? __ldcg(keys + s_cand[i]) : 0u;
+        const unsigned o = i < static_cast<int>(nc) ? (ckey ? s_ckey[i] : __ldcg(keys + s_cand[i])) : 0u;
         const unsigned gt = i < static_cast<int>(nc) && o > thr, eq = i < static_cast<int>(nc) && o == thr;
         const unsigned packed = (gt << 16) | eq;
         const unsigned incl = block_inclusive_scan(packed, s_warp);
@@ -2506,8 +2530,12 @@ __global__ void __launch_bounds__(kBudgetThreads) k_budget(DevParams P) {
   grid_dependency_wait();
   const int u = blockIdx.x;
   const UnitInfo inf = P.info[u];
+  const float* ps = P.pscore + static_cast<size_t>(u) * P.max_ctx * G;
+  // the scores' first batch is in flight while the maxima are found
+  float first[kBudgetBatch][G];
+  load_budget_batch<G>(ps, inf.mode == 2 ? inf.nI + inf.p : 0, first);
   if (inf.mode == 2) det_record_max<D, G>(P, u, s_mh);
-  unit_budget<G>(P, u, inf, P.pscore + static_cast<size_t>(u) * P.max_ctx * G, s_mh);
+  unit_budget<G>(P, u, inf, ps, s_mh, first);
   grid_dependents_launch();
 }
 
