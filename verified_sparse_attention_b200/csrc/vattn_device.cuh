@@ -298,61 +298,10 @@ __device__ __forceinline__ unsigned block_inclusive_scan(unsigned v, unsigned* s
   return v + base;
 }
 
-__device__ __forceinline__ unsigned block_sum(unsigned v, unsigned* s_warp) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) s_warp[warp] = v;
-  __syncthreads();
-  unsigned tot = 0;
-  for (int i = 0; i < nw; i++) tot += s_warp[i];
-  __syncthreads();
-  return tot;
-}
-
-// Radix-select step over a histogram: find the bin holding the krem-th largest
-// key (counting from the top bin) and the rank left inside that bin.
-// Block of 256 threads; NB a multiple of 1024 (each thread reads NB/256 bins
-// with 16-byte loads, all issued before use).
-template <int NB>
-__device__ __forceinline__ void find_digit(const unsigned* __restrict__ hist, int krem,
-                                           int* s_digit, int* s_krem, unsigned* s_warp) {
-  constexpr int PER = NB / 256;
-  static_assert(PER % 4 == 0, "bins per thread must fill 16-byte loads");
-  const int t = threadIdx.x;
-  const int lo = NB - (t + 1) * PER;  // this thread's bins are [lo, lo + PER), scanned downwards
-  unsigned v[PER];
-#pragma unroll
-  for (int i = 0; i < PER / 4; i++) {
-    const uint4 w = *reinterpret_cast<const uint4*>(hist + lo + 4 * i);
-    v[4 * i] = w.x;
-    v[4 * i + 1] = w.y;
-    v[4 * i + 2] = w.z;
-    v[4 * i + 3] = w.w;
-  }
-  unsigned sum = 0;
-#pragma unroll
-  for (int i = 0; i < PER; i++) sum += v[i];
-  const unsigned incl = block_inclusive_scan(sum, s_warp);
-  const unsigned excl = incl - sum;
-  if (excl < static_cast<unsigned>(krem) && static_cast<unsigned>(krem) <= incl) {
-    unsigned c = excl;
-    bool done = false;
-#pragma unroll
-    for (int i = PER - 1; i >= 0; i--) {
-      if (!done && c + v[i] >= static_cast<unsigned>(krem)) {
-        *s_digit = lo + i;
-        *s_krem = krem - static_cast<int>(c);
-        done = true;
-      }
-      c += v[i];
-    }
-  }
-  __syncthreads();
-}
-
-// find_digit for any block of BT threads over a shared-memory histogram
-// (each thread scans NB / BT consecutive bins downwards).
+// Radix-select step over a shared-memory histogram, for any block of BT
+// threads: find the bin holding the krem-th largest key (counting from the
+// top bin) and the rank left inside that bin; each thread scans NB / BT
+// consecutive bins downwards.
 template <int NB, int BT>
 __device__ __forceinline__ void find_digit_bt(const unsigned* hist, int krem, int* s_digit, int* s_krem,
                                               unsigned* s_warp) {
